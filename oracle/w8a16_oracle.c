@@ -1,0 +1,241 @@
+/*
+ * CPU oracle for the W8A16 linear layer -- TEST INFRASTRUCTURE ONLY.
+ *
+ * This file is the plain, slow, obviously-correct restatement of what the
+ * GPU path computes.  Only the test-suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load it; the product library never links
+ * or calls it, and it shares no code, header or table with the CUDA path.
+ *
+ * Sources (web pages on int8 weight-only quantization):
+ *  - TPU-MLIR ChatGLM2 W8A16 article ("Exploring INT8 deployment of ChatGLM2
+ *    on BM1684X"), section 2 "quantization scheme": only the Linear-layer
+ *    weights are quantized, per channel, to int8; at compute time they are
+ *    dequantized back to F16; activations stay F16.
+ *  - same article, section 3 "TPU-MLIR implementation": the weight
+ *    R = 4096x27392 F16 becomes int8 plus an F16 scale vector.
+ *  - same article, section 4 "backend performance": the op loads, casts
+ *    INT8 to F16, multiplies by the scale, multiplies with the activation
+ *    and stores the result (steps 1-5).
+ *  - LightSeq 2020 slides, slides "quantization: clipping + symmetric":
+ *    symmetric quantization with bound = max|W| and 2^(n-1)-1 = 127 levels
+ *    on each side of zero.
+ * Where the pages leave a step open the following readings are used (each
+ * is listed with its reason in the design notes):
+ *  - one scale per OUTPUT channel n (column of W[K,N]);
+ *  - scale_n = fp16_rne( fp32( amax_n / 127 ) ), the division in IEEE fp32;
+ *  - q = clamp( rne( W / s ), -127, 127 ) with s the STORED fp16 scale
+ *    widened to fp32, the division in IEEE fp32, ties to even;
+ *  - an all-zero column has s = +0 and q = 0;
+ *  - Y = X . (q o s) computed in the factored form s_n * sum_k x_k q_kn
+ *    (exact in real arithmetic), here in fp64, plus an optional fp16 bias;
+ *    the result is returned in fp64 and NOT rounded to fp16.
+ * Inputs are assumed finite (NaN/Inf in W or X are outside the contract).
+ *
+ * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -fPIC -shared
+ * (no SIMD intrinsics, no threads, no blocking).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------------
+ * IEEE-754 binary16 <-> binary32, written from the format definition
+ * (1 sign bit, 5 exponent bits with bias 15, 10 fraction bits; subnormals
+ * kept; round to nearest, ties to even).
+ * ------------------------------------------------------------------- */
+
+float oracle_f16_to_f32(uint16_t h)
+{
+    uint32_t sign = (uint32_t)(h >> 15) & 1u;
+    uint32_t exp = (uint32_t)(h >> 10) & 0x1Fu;
+    uint32_t frac = (uint32_t)h & 0x3FFu;
+    float mag;
+    if (exp == 0) {
+        /* zero or subnormal: frac * 2^-24, exact in binary32 */
+        mag = ldexpf((float)frac, -24);
+    } else if (exp == 31) {
+        mag = frac ? NAN : INFINITY;
+    } else {
+        /* (1024 + frac) * 2^(exp - 25), exact in binary32 */
+        mag = ldexpf((float)(1024u + frac), (int)exp - 25);
+    }
+    return sign ? -mag : mag;
+}
+
+uint16_t oracle_f32_to_f16(float f)
+{
+    uint32_t x;
+    memcpy(&x, &f, sizeof x);
+    uint16_t sign = (uint16_t)((x >> 16) & 0x8000u);
+    uint32_t exp32 = (x >> 23) & 0xFFu;
+    uint32_t man32 = x & 0x7FFFFFu;
+
+    if (exp32 == 0xFFu) {                      /* Inf or NaN */
+        return (uint16_t)(sign | 0x7C00u | (man32 ? 0x200u : 0u));
+    }
+    if (exp32 == 0 && man32 == 0) {
+        return sign;                          /* signed zero */
+    }
+    /* value = m * 2^e with m an integer (24-bit for normals) */
+    int32_t e;
+    uint32_t m;
+    if (exp32 == 0) {                          /* binary32 subnormal */
+        m = man32;
+        e = -149;
+    } else {
+        m = man32 | 0x800000u;
+        e = (int32_t)exp32 - 150;
+    }
+    /* Target: binary16 value = M * 2^E, where for normals 1024 <= M < 2048
+     * and E = exponent - 25 >= -24; subnormals have E = -24, M < 1024.
+     * Find the binary16 exponent of |f|: floor(log2(m * 2^e)). */
+    int32_t msb = 31;
+    while (((m >> msb) & 1u) == 0u) {
+        msb--;
+    }
+    int32_t log2v = msb + e;                   /* floor(log2 |f|) */
+    int32_t E = log2v - 10;                    /* ulp exponent for a normal */
+    if (E < -24) {
+        E = -24;                               /* subnormal range: ulp 2^-24 */
+    }
+    /* M = round_half_even(m * 2^(e - E)) */
+    int32_t shift = E - e;                     /* bits to drop (may be <= 0) */
+    uint64_t M;
+    if (shift <= 0) {
+        M = (uint64_t)m << (uint32_t)(-shift);
+    } else if (shift >= 40) {
+        M = 0;                                 /* far below half an ulp */
+    } else {
+        uint64_t mm = m;
+        uint64_t q = mm >> (uint32_t)shift;
+        uint64_t rem = mm & ((1ull << (uint32_t)shift) - 1ull);
+        uint64_t half = 1ull << (uint32_t)(shift - 1);
+        if (rem > half || (rem == half && (q & 1ull))) {
+            q += 1;
+        }
+        M = q;
+    }
+    /* Rounding may carry into the next binade. */
+    if (M >= 2048u) {
+        M >>= 1;
+        E += 1;
+    }
+    if (M >= 1024u) {
+        int32_t biased = E + 25;               /* exponent field */
+        if (biased >= 31) {
+            return (uint16_t)(sign | 0x7C00u);  /* overflow -> Inf */
+        }
+        return (uint16_t)(sign | ((uint32_t)biased << 10) | ((uint32_t)M - 1024u));
+    }
+    /* subnormal (E == -24), or zero after rounding */
+    return (uint16_t)(sign | (uint32_t)M);
+}
+
+/* ---------------------------------------------------------------------
+ * Per-output-channel symmetric int8 quantization of W[K,N] (row-major).
+ * Step order as the pages give it: bound = max|W| over the channel, the
+ * scale puts the bound on level 127, then every weight is divided by the
+ * scale, rounded and clipped to the symmetric range.
+ * ------------------------------------------------------------------- */
+
+static void quantize_column(const float *col_vals, int64_t K, int8_t *q_col,
+                            int64_t N, uint16_t *scale_out)
+{
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf(col_vals[k]);
+        if (a > amax) {
+            amax = a;
+        }
+    }
+    float s32 = amax / 127.0f;                 /* IEEE fp32 division */
+    uint16_t s16 = oracle_f32_to_f16(s32);
+    float s = oracle_f16_to_f32(s16);
+    for (int64_t k = 0; k < K; ++k) {
+        int32_t qi;
+        if (s == 0.0f) {
+            qi = 0;
+        } else {
+            float r = col_vals[k] / s;         /* IEEE fp32 division */
+            float rr = nearbyintf(r);          /* default mode: ties to even */
+            if (rr > 127.0f) {
+                rr = 127.0f;
+            }
+            if (rr < -127.0f) {
+                rr = -127.0f;
+            }
+            qi = (int32_t)rr;
+        }
+        q_col[k * N] = (int8_t)qi;
+    }
+    *scale_out = s16;
+}
+
+/* W fp32 [K,N] -> q int8 [K,N], scales fp16 bits [N].  col_buf: K floats. */
+void oracle_quantize_f32(const float *W, int64_t K, int64_t N, int8_t *q,
+                         uint16_t *scales, float *col_buf)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            col_buf[k] = W[k * N + n];
+        }
+        quantize_column(col_buf, K, q + n, N, &scales[n]);
+    }
+}
+
+/* W fp16 bits [K,N]: widened exactly to fp32, then as above. */
+void oracle_quantize_f16(const uint16_t *W, int64_t K, int64_t N, int8_t *q,
+                         uint16_t *scales, float *col_buf)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            col_buf[k] = oracle_f16_to_f32(W[k * N + n]);
+        }
+        quantize_column(col_buf, K, q + n, N, &scales[n]);
+    }
+}
+
+/* ---------------------------------------------------------------------
+ * Y[M,N] = X[M,K] . dequant(q)[K,N] (+ bias), in fp64.
+ *   Y[m,n] = s_n * sum_k X[m,k] * q[k,n] + bias_n
+ * acc: N doubles of caller-provided scratch.  bias may be NULL.
+ * ------------------------------------------------------------------- */
+void oracle_linear(const uint16_t *X, const int8_t *q, const uint16_t *scales,
+                   const uint16_t *bias, int64_t M, int64_t K, int64_t N,
+                   double *Y, double *acc)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            acc[n] = 0.0;
+        }
+        for (int64_t k = 0; k < K; ++k) {
+            double x = (double)oracle_f16_to_f32(X[m * K + k]);
+            const int8_t *qrow = q + k * N;
+            for (int64_t n = 0; n < N; ++n) {
+                acc[n] += x * (double)qrow[n];
+            }
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double y = acc[n] * (double)oracle_f16_to_f32(scales[n]);
+            if (bias) {
+                y += (double)oracle_f16_to_f32(bias[n]);
+            }
+            Y[m * N + n] = y;
+        }
+    }
+}
+
+/* Element-wise array forms of the two conversions (used by the pins). */
+void oracle_f32_to_f16_array(const float *src, int64_t n, uint16_t *dst)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        dst[i] = oracle_f32_to_f16(src[i]);
+    }
+}
+
+void oracle_f16_to_f32_array(const uint16_t *src, int64_t n, float *dst)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        dst[i] = oracle_f16_to_f32(src[i]);
+    }
+}

@@ -1,0 +1,74 @@
+"""Plant plausible mistakes in copies of the CPU oracle and check that the
+pins catch every one of them (mutation testing, CPU only).
+
+Each mutant is the oracle's C source with one textual change, compiled to a
+temporary shared library.  A mutant "survives" if every pin still passes.
+"""
+import os
+import tempfile
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+MUTANTS = {
+    # quantization
+    "scale_over_128": ("amax / 127.0f", "amax / 128.0f"),
+    "round_half_away": ("nearbyintf(r)", "roundf(r)"),
+    "truncate": ("nearbyintf(r)", "truncf(r)"),
+    "divide_by_fp32_scale": ("float r = col_vals[k] / s;", "float r = col_vals[k] / s32;"),
+    "clip_to_minus_128": ("if (rr < -127.0f) {\n                rr = -127.0f;",
+                          "if (rr < -128.0f) {\n                rr = -128.0f;"),
+    "no_abs_in_bound": ("float a = fabsf(col_vals[k]);", "float a = col_vals[k];"),
+    "bound_skips_first_row": ("    for (int64_t k = 0; k < K; ++k) {\n        float a",
+                              "    for (int64_t k = 1; k < K; ++k) {\n        float a"),
+    # fp16 codec
+    "f16_ties_away": ("(rem == half && (q & 1ull))", "(rem == half)"),
+    "f16_flush_subnormals": ("    return (uint16_t)(sign | (uint32_t)M);\n}",
+                             "    return (uint16_t)(sign);\n}"),
+    "f16_exponent_off_by_one": ("int32_t biased = E + 25;", "int32_t biased = E + 24;"),
+    # linear
+    "drop_scale": ("double y = acc[n] * (double)oracle_f16_to_f32(scales[n]);",
+                   "double y = acc[n];"),
+    "bias_subtracted": ("y += (double)oracle_f16_to_f32(bias[n]);",
+                        "y -= (double)oracle_f16_to_f32(bias[n]);"),
+    "transposed_weight_index": ("acc[n] += x * (double)qrow[n];",
+                                "acc[n] += x * (double)q[n * K + k];"),
+    "x_row_ignored": ("oracle_f16_to_f32(X[m * K + k])", "oracle_f16_to_f32(X[k])"),
+    "scale_indexed_by_row": ("(double)oracle_f16_to_f32(scales[n]);",
+                             "(double)oracle_f16_to_f32(scales[m]);"),
+}
+
+
+def _compile_mutant(name, old, new, tmpdir):
+    with open(oracle._SRC) as f:
+        src = f.read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique/found"
+    path = os.path.join(tmpdir, f"{name}.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    so = os.path.join(tmpdir, f"lib{name}.so")
+    oracle.build(force=True, src=path, out=so)
+    return oracle.Oracle(so)
+
+
+@pytest.fixture(scope="module")
+def tmpdir():
+    with tempfile.TemporaryDirectory() as d:
+        yield d
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_kill_mutant(name, tmpdir):
+    old, new = MUTANTS[name]
+    orc = _compile_mutant(name, old, new, tmpdir)
+    killed = []
+    for pin in pins.PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(orc)
+        except (AssertionError, ValueError, IndexError):
+            killed.append(pin.__name__)
+    assert killed, f"mutant {name} survived every pin"

@@ -1,0 +1,313 @@
+"""Pins for the CPU oracle: checks against what the pages and mathematics fix,
+never against a retyped copy of the oracle's own formula.
+
+Sources: TPU-MLIR ChatGLM2 W8A16 article (sections 2-4) and LightSeq 2020
+slides ("quantization: clipping + symmetric").
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+from tests import golden
+
+SEED = synthetic.SEED
+
+
+# ---------------------------------------------------------------- fp16 codec
+# Pinned to numpy's IEEE binary16 conversion (a library routine).
+
+def pin_f16_to_f32_every_pattern(orc):
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = orc.f16_bits_to_f32(h)
+    ref = h.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def pin_f32_to_f16_round_trips_every_fp16_value(orc):
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f = h.view(np.float16)
+    keep = ~np.isnan(f)
+    back = orc.f32_to_f16_bits(f[keep].astype(np.float32))
+    assert np.array_equal(back, h[keep])
+
+
+def pin_f32_to_f16_ties_go_to_even(orc):
+    # midpoints between adjacent finite fp16 values (exact in fp32)
+    h = np.arange(0, 0x7BFF, dtype=np.uint16)
+    lo = h.view(np.float16).astype(np.float64)
+    hi = (h + 1).view(np.float16).astype(np.float64)
+    mid = ((lo + hi) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (lo + hi) / 2)
+    got = orc.f32_to_f16_bits(mid)
+    assert np.all(got % 2 == 0)                     # even significand
+    assert np.all((got == h) | (got == h + 1))
+    assert np.array_equal(got, mid.astype(np.float16).view(np.uint16))
+    got_neg = orc.f32_to_f16_bits(-mid)
+    assert np.array_equal(got_neg, got | np.uint16(0x8000))
+
+
+def pin_f32_to_f16_random_against_numpy(orc):
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, 1 << 32, size=2_000_000, dtype=np.uint64).astype(np.uint32)
+    f = bits.view(np.float32)
+    f = f[np.isfinite(f)]
+    # also a dense sample around the fp16 range, including fp16 subnormals
+    g = (rng.standard_normal(1_000_000) * np.exp(rng.uniform(-20, 12, 1_000_000))).astype(np.float32)
+    for x in (f, g):
+        got = orc.f32_to_f16_bits(x)
+        ref = x.astype(np.float16).view(np.uint16)
+        assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------------ quantization
+
+def _wq(K, N, tid, outliers=0.001):
+    return synthetic.weights(K, N, SEED, tid, outlier_frac=outliers)
+
+
+def pin_symmetric_levels_from_slides(orc):
+    g = golden.load("symmetric_levels.txt")
+    top = 2 ** (g["bits"] - 1) - 1
+    assert top == g["top_level"] == 127
+    W = _wq(300, 264, 11)
+    q, s = orc.quantize(W)
+    assert q.min() >= -top and q.max() <= top
+    assert not np.any(q == -128)
+    # the bound max|W| of every channel lands on the top level, with its sign
+    arg = np.argmax(np.abs(W), axis=0)
+    cols = np.arange(W.shape[1])
+    assert np.all(np.abs(q[arg, cols]) == top)
+    assert np.all(np.sign(q[arg, cols]) == np.sign(W[arg, cols]))
+
+
+def pin_error_bound_half_a_step(orc):
+    # |w - q s| <= s/2, up to the single fp32 rounding of w/s
+    for tid, (K, N) in enumerate([(300, 264), (64, 8), (1, 16), (1000, 40)]):
+        W = _wq(K, N, 20 + tid)
+        q, s = orc.quantize(W)
+        s64 = s.astype(np.float64)
+        err = np.abs(W.astype(np.float64) - q.astype(np.float64) * s64)
+        assert np.all(err <= s64 * (0.5 + 2.0 ** -16))
+
+
+def pin_scale_is_fp16_of_fp32_amax_over_127(orc):
+    # library pin: numpy fp32 division (IEEE) then numpy fp16 rounding
+    W = _wq(257, 72, 30)
+    _, s = orc.quantize(W)
+    amax = np.max(np.abs(W), axis=0).astype(np.float32)
+    ref = (amax / np.float32(127.0)).astype(np.float16)
+    assert np.array_equal(s.view(np.uint16), ref.view(np.uint16))
+
+
+def pin_exact_multiples_round_trip(orc):
+    rng = np.random.default_rng(5)
+    K, N = 200, 12
+    for s0 in [2.0 ** -10, 0.0004506, 1.5e-3, 0.0078125, 3.0]:
+        s0 = float(np.float16(s0))
+        j = rng.integers(-127, 128, size=(K, N))
+        j[rng.integers(0, K, size=N), np.arange(N)] = rng.choice([-127, 127], size=N)
+        W = (j * s0).astype(np.float32)
+        assert np.array_equal(W.astype(np.float64), j * s0)        # exact
+        q, s = orc.quantize(W)
+        assert np.all(s.astype(np.float64) == s0)
+        assert np.array_equal(q.astype(np.int64), j)
+
+
+def pin_ties_round_half_to_even(orc):
+    js = np.arange(-126, 126)
+    for s0 in [2.0 ** -8, float(np.float16(0.0123))]:
+        col = np.concatenate([[127.0 * s0], (js + 0.5) * s0]).astype(np.float32)
+        assert np.array_equal(col[1:].astype(np.float64), (js + 0.5) * s0)
+        q, s = orc.quantize(col.reshape(-1, 1))
+        assert float(s[0]) == s0
+        got = q[1:, 0].astype(np.int64)
+        want = np.where(js % 2 == 0, js, js + 1)         # nearest even integer
+        assert np.array_equal(got, want)
+
+
+def pin_subnormal_scale_clamps_to_symmetric_range(orc):
+    # A channel whose scale is an fp16 subnormal is coarsely rounded: here
+    # s32 = 1.4 * 2^-24 rounds to s = 2^-24, so amax/s is about 178 and the
+    # clip must hold the codes at +-127 (never -128).
+    amax = np.float32(127 * 1.4 * 2.0 ** -24)
+    col = np.array([amax, -amax, amax / 2, np.float32(3 * 2.0 ** -24)], dtype=np.float32)
+    q, s = orc.quantize(np.stack([col, -col], axis=1))
+    assert np.all(s.view(np.uint16) == 1)                  # 2^-24
+    assert q[0, 0] == 127 and q[1, 0] == -127 and q[0, 1] == -127 and q[1, 1] == 127
+    assert q[3, 0] == 3 and q[3, 1] == -3
+
+
+def pin_zero_column_has_zero_scale_and_codes(orc):
+    W = _wq(64, 16, 40)
+    W[:, 3] = 0.0
+    W[:, 9] = -0.0
+    q, s = orc.quantize(W)
+    assert s.view(np.uint16)[3] == 0 and s.view(np.uint16)[9] == 0
+    assert not np.any(q[:, 3]) and not np.any(q[:, 9])
+
+
+def pin_divides_by_the_stored_fp16_scale(orc):
+    # Reading of the pages: the weights are divided by the scale that is
+    # stored (fp16), so that q*s reconstructs w within s/2 for the shipped s.
+    amax = np.float32(1.0)
+    s32 = amax / np.float32(127.0)
+    s16 = np.float32(np.float16(s32))
+    assert s16 != s32
+    w = np.float32(100.502) * s16
+    by16 = np.rint(w / s16)
+    by32 = np.rint(w / s32)
+    assert by16 != by32                         # the case distinguishes them
+    q, s = orc.quantize(np.array([[amax], [w]], dtype=np.float32))
+    assert np.float32(s[0]) == s16
+    assert q[1, 0] == by16
+
+
+def pin_per_channel_independence(orc):
+    W = _wq(128, 32, 50)
+    q, s = orc.quantize(W)
+    W2 = W.copy()
+    W2[:, 5] *= np.float32(4.0)                 # power of two: exact
+    q2, s2 = orc.quantize(W2)
+    assert np.array_equal(q, q2)
+    assert float(s2[5]) == 4.0 * float(s[5])
+    keep = np.arange(32) != 5
+    assert np.array_equal(s[keep].view(np.uint16), s2[keep].view(np.uint16))
+
+
+def pin_fp16_weights_match_widened_fp32(orc):
+    W16 = _wq(96, 40, 60).astype(np.float16)
+    qa, sa = orc.quantize(W16)
+    qb, sb = orc.quantize(W16.astype(np.float32))
+    assert np.array_equal(qa, qb)
+    assert np.array_equal(sa.view(np.uint16), sb.view(np.uint16))
+
+
+def pin_codes_are_the_nearest_level_by_brute_force(orc):
+    # Independent characterisation: among all 255 levels, q is the one
+    # nearest to the fp32 quotient w/s (ties to the even level).
+    W = _wq(9, 6, 70)
+    q, s = orc.quantize(W)
+    for n in range(W.shape[1]):
+        sn = np.float32(s[n])
+        for k in range(W.shape[0]):
+            r = Fraction(float(np.float32(W[k, n]) / sn))
+            best = None
+            for lv in range(-127, 128):
+                d = abs(r - lv)
+                if best is None or d < best[0] or (d == best[0] and lv % 2 == 0):
+                    best = (d, lv)
+            assert q[k, n] == best[1]
+
+
+def pin_weight_bytes_halve_as_printed(orc):
+    g = golden.load("chatglm2_h_to_4h_weight_bytes.txt")
+    K, N = g["K"], g["N"]
+    f16_bytes = K * N * np.dtype(np.float16).itemsize
+    # quantized storage of a small slab scales linearly: 1 byte per weight
+    q, s = orc.quantize(_wq(64, 128, 80))
+    per_weight = q.nbytes / q.size
+    int8_bytes = K * N * per_weight
+    assert round(f16_bytes / 2 ** 20) == g["f16_mb"]
+    assert round(int8_bytes / 2 ** 20) == g["int8_mb"]
+    # the printed scale vector has 4096 f16 entries = 0.008 MB
+    assert round(g["scale_entries_printed"] * 2 / 2 ** 20, 3) == g["scale_mb_printed"]
+    # one fp16 scale per output channel (the reading used here) costs N*2
+    # bytes, still well under 0.1 % of the int8 weight
+    scale_bytes = N * s.itemsize
+    assert scale_bytes / int8_bytes < 1e-3
+
+
+# ------------------------------------------------------------------ linear
+
+def pin_linear_exact_on_integer_inputs(orc):
+    # Integer X, power-of-two scales: the exact result is an integer matmul
+    # (numpy int64) times the scale, with no rounding anywhere.
+    rng = np.random.default_rng(7)
+    M, K, N = 5, 96, 40
+    Xi = rng.integers(-8, 9, size=(M, K))
+    qi = rng.integers(-127, 128, size=(K, N)).astype(np.int8)
+    s = (2.0 ** rng.integers(-12, -2, size=N)).astype(np.float16)
+    b = (rng.integers(-64, 64, size=N) / 16.0).astype(np.float16)
+    Y = orc.linear(Xi.astype(np.float16), qi, s, b)
+    exact = (Xi @ qi.astype(np.int64)) * s.astype(np.float64) + b.astype(np.float64)
+    assert np.array_equal(Y, exact)
+    Y0 = orc.linear(Xi.astype(np.float16), qi, s, None)
+    assert np.array_equal(Y0, (Xi @ qi.astype(np.int64)) * s.astype(np.float64))
+
+
+def pin_linear_unit_vectors_select_rows(orc):
+    rng = np.random.default_rng(8)
+    K, N = 33, 24
+    q = rng.integers(-127, 128, size=(K, N)).astype(np.int8)
+    s = (rng.uniform(1e-4, 1e-2, N)).astype(np.float16)
+    ks = [0, 7, 32]
+    X = np.zeros((len(ks), K), dtype=np.float16)
+    X[np.arange(len(ks)), ks] = 1.0
+    Y = orc.linear(X, q, s)
+    for m, k in enumerate(ks):
+        assert np.array_equal(Y[m], q[k].astype(np.float64) * s.astype(np.float64))
+
+
+def pin_linear_against_exact_rationals(orc):
+    X = synthetic.activations(2, 5, SEED, 91)
+    q = np.array([[3, -127, 0], [127, 5, -6], [-1, 2, 99], [64, -64, 1], [0, 0, -7]], dtype=np.int8)
+    s = np.array([0.001, 0.0625, 3.5e-4], dtype=np.float16)
+    b = np.array([0.5, -0.25, 0.0], dtype=np.float16)
+    Y = orc.linear(X, q, s, b)
+    for m in range(2):
+        for n in range(3):
+            acc = sum(Fraction(float(X[m, k])) * int(q[k, n]) for k in range(5))
+            exact = acc * Fraction(float(s[n])) + Fraction(float(b[n]))
+            assert abs(Fraction(Y[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 50)
+
+
+def pin_linear_matches_numpy_matmul(orc):
+    M, K, N = 4, 256, 512
+    W = synthetic.weights(K, N, SEED, 101)
+    X = synthetic.activations(M, K, SEED, 102)
+    b = synthetic.bias(N, SEED, 103)
+    q, s = orc.quantize(W)
+    Y = orc.linear(X, q, s, b)
+    ref = X.astype(np.float64) @ (q.astype(np.float64) * s.astype(np.float64)) + b.astype(np.float64)
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_cosine_similarity_as_printed(orc):
+    g = golden.load("w8a16_cosine.txt")
+    K, N, M = 4096, 256, 4
+    W = synthetic.weights(K, N, SEED, 111, outlier_frac=0.001)
+    X = synthetic.activations(M, K, SEED, 112)
+    q, s = orc.quantize(W)
+    Yq = orc.linear(X, q, s).ravel()
+    Yf = (X.astype(np.float64) @ W.astype(np.float64)).ravel()
+    cos = float(Yq @ Yf / (np.linalg.norm(Yq) * np.linalg.norm(Yf)))
+    assert cos > g["min_cosine"]
+
+
+def pin_tolerance_helper_rejects_a_planted_error(orc):
+    M, K, N = 4, 256, 512
+    q, s = orc.quantize(synthetic.weights(K, N, SEED, 121))
+    X = synthetic.activations(M, K, SEED, 122)
+    Y = orc.linear(X, q, s)
+    Y16 = Y.astype(np.float16).astype(np.float64)
+    assert oracle.tolerance_ok(Y16, Y)[0]
+    bad = Y16.copy()
+    bad[1, 7] += 4e-3 * np.abs(Y).max()
+    assert not oracle.tolerance_ok(bad, Y)[0]
+    # a dropped scale on one channel is caught
+    s_bad = s.copy()
+    s_bad[3] = np.float16(float(s[3]) * 1.01)
+    assert not oracle.tolerance_ok(orc.linear(X, q, s_bad), Y)[0]
+
+
+PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__[4:] for p in PINS])
+def test_oracle_pin(pin):
+    pin(oracle.default())
