@@ -1,0 +1,182 @@
+/*
+ * w8a16.h -- C ABI of libw8a16.so, a W8A16 (int8 weight, fp16 activation)
+ * linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The operation (TPU-MLIR ChatGLM2 W8A16 article, section 2 "quantization
+ * scheme" and section 4 "backend performance", steps 1-5; LightSeq 2020
+ * slides "quantization: clipping + symmetric"):
+ *
+ *   quantize   s_n = fp16_rne( fp32(max_k |W[k,n]|) / 127 )          (per n)
+ *              q[k,n] = clamp( rne( W[k,n] / float(s_n) ), -127, 127 )
+ *              (s_n == 0 for an all-zero column, and then q = 0)
+ *   linear     Y[m,n] = fp16_rne( s_n * sum_k X[m,k] * q[k,n] + bias_n )
+ *              with the sum accumulated in fp32.
+ *
+ * The page dequantizes the weight (cast int8 -> F16, multiply by the scale)
+ * before the matmul; here the per-channel scale is applied once per output
+ * element after the sum, which is the same value in exact arithmetic.
+ *
+ * Conventions for every entry point
+ *  - Tensors are dense row-major.  W and q are [K, N] (K = input features,
+ *    the reduction dimension; N = output features / channels, contiguous).
+ *    X is [M, K], Y is [M, N], scales and bias are [N].
+ *  - fp16 buffers are passed as uint16_t* holding IEEE binary16 bit patterns.
+ *  - Every pointer except `bias` (nullable) and host-side outputs is a
+ *    DEVICE pointer on the current CUDA device and must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work on that stream; they never allocate
+ *    device memory and never synchronize (except the diagnostic
+ *    w8_device_status).  The caller owns every buffer.
+ *  - Invalid arguments are detected on the host before anything is launched
+ *    and reported by a negative w8_status; nothing is written then.  A
+ *    launch failure is W8_ERR_CUDA.  Errors raised while a kernel runs
+ *    surface at the caller's next synchronization.
+ *  - Every wait inside a kernel is bounded (about one second); a wait that
+ *    runs out records a status word readable with w8_device_status() and the
+ *    kernel returns early instead of hanging.
+ *  - The library keeps no per-call state.  It is safe to call from several
+ *    host threads on different streams, provided calls that share a
+ *    workspace do not overlap on the device.
+ */
+#ifndef W8A16_H
+#define W8A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W8_OK = 0,
+    W8_ERR_NULL = -1,       /* a required pointer is NULL */
+    W8_ERR_SHAPE = -2,      /* a size is out of range or not a multiple of 8 */
+    W8_ERR_ALIGN = -3,      /* a pointer is not 16-byte aligned */
+    W8_ERR_DTYPE = -4,      /* unknown w8_dtype */
+    W8_ERR_WORKSPACE = -5,  /* workspace missing or smaller than required */
+    W8_ERR_CUDA = -6,       /* a CUDA runtime call or launch failed */
+    W8_ERR_TIMEOUT = -7,    /* a bounded device wait ran out (see w8_device_status) */
+    W8_ERR_ALIAS = -8,      /* the output overlaps an input */
+    W8_ERR_DEVICE = -9      /* the current device is not sm_100 */
+} w8_status;
+
+typedef enum { W8_F32 = 0, W8_F16 = 1 } w8_dtype;
+
+/* Tile geometry of the packed weight layout (see w8_prepack). */
+#define W8_TILE_N 128
+#define W8_TILE_K 64
+#define W8_TILE_BYTES (W8_TILE_N * W8_TILE_K)
+
+/*
+ * w8_quantize_per_channel -- per-output-channel symmetric int8 quantization
+ * (the weight quantizer of the TPU-MLIR article, section 3: a 2-D weight
+ * R = 4096 x 27392 becomes int8 plus an F16 scale per channel).
+ *
+ *   W       [K, N] input weight, fp32 or fp16 as given by w_dtype (W8_F32 /
+ *           W8_F16); fp16 is widened exactly to fp32 first.
+ *   q       [K, N] int8 output codes in [-127, 127].
+ *   scales  [N] fp16 output scales.
+ *   K >= 1; N >= 0 with N % 8 == 0 (N == 0 is a no-op).
+ * The result is bit-exact: fp32 divisions are IEEE round-to-nearest, the
+ * fp32 -> fp16 and fp32 -> int conversions round half to even, fp16
+ * subnormal scales are kept.  Inputs must be finite.
+ * Errors: W8_ERR_NULL, W8_ERR_SHAPE, W8_ERR_ALIGN, W8_ERR_DTYPE,
+ *         W8_ERR_ALIAS (q overlaps W), W8_ERR_CUDA.
+ */
+int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N,
+                            int8_t *q, uint16_t *scales, void *stream);
+
+/*
+ * w8_prepacked_bytes -- size of the packed weight for a [K, N] q:
+ * ceil(N/128) * ceil(K/64) * 8192 bytes (== K*N when K % 64 == 0 and
+ * N % 128 == 0).  Returns 0 for K < 1 or N < 1.
+ */
+size_t w8_prepacked_bytes(int64_t K, int64_t N);
+
+/*
+ * w8_prepack -- reorder q [K, N] into the tiled layout both linear kernels
+ * stream (done once per weight, off the per-call path).
+ *
+ * Layout: tiles of 128 output channels x 64 input features, 8192 bytes
+ * each.  Tile (b, kb) -- channels n in [128b, 128b+128), features k in
+ * [64kb, 64kb+64) -- starts at byte (b * ceil(K/64) + kb) * 8192, so the
+ * tiles of one channel block are contiguous along K.  Inside a tile, row r
+ * (channel n = 128b + r) takes bytes [64r, 64r + 64); its 16-byte chunk c
+ * (features 64kb + 16c ... +15, in natural order) is stored at chunk slot
+ * c XOR ((r >> 1) & 3).  Each byte holds q + 128 (offset binary, i.e.
+ * q XOR 0x80).  Positions with k >= K or n >= N hold 0x80 (q = 0).
+ *   q       [K, N] int8 input; packed: w8_prepacked_bytes(K, N) output bytes.
+ *   K >= 1, N >= 1, N % 8 == 0.
+ * Errors: W8_ERR_NULL, W8_ERR_SHAPE, W8_ERR_ALIGN, W8_ERR_ALIAS, W8_ERR_CUDA.
+ */
+int w8_prepack(const int8_t *q, int64_t K, int64_t N, uint8_t *packed, void *stream);
+
+/*
+ * w8_unpack -- inverse of w8_prepack (packed -> q [K, N]); for tests and
+ * inspection.  Same argument rules as w8_prepack.
+ */
+int w8_unpack(const uint8_t *packed, int64_t K, int64_t N, int8_t *q, void *stream);
+
+/*
+ * w8a16_workspace_bytes -- device scratch w8a16_linear needs for this shape
+ * on the CURRENT device (it depends on the SM count).  0 means none.  The
+ * decode path (M <= 16) splits the reduction over K across thread blocks
+ * and needs room for fp32 partial sums plus one int32 counter per 128
+ * output channels.
+ */
+size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
+
+/*
+ * w8a16_linear -- Y = X . dequant(packed, scales) (+ bias).
+ *
+ *   X          [M, K] fp16 activations.
+ *   packed     w8_prepack output for the [K, N] weight.
+ *   scales     [N] fp16 per-channel scales (w8_quantize_per_channel output).
+ *   bias       [N] fp16 or NULL.
+ *   Y          [M, N] fp16 output; must not overlap X, packed or scales.
+ *   M >= 0 (0 is a no-op); K >= 1 with K % 8 == 0; N >= 1 with N % 8 == 0.
+ *   workspace  device scratch of at least w8a16_workspace_bytes(M, K, N)
+ *              bytes (may be NULL when that is 0).  It must be all zero
+ *              before its first use; every call leaves it ready for the
+ *              next one.  Calls sharing one workspace must not run
+ *              concurrently on the device.
+ * Kernel choice (internal): M <= 16 streams the weight once with a
+ * split-K decode kernel (HBM-bound); larger M runs a tcgen05 tensor-core
+ * kernel with the widened weight tile held in tensor memory.
+ * Accuracy: |Y - Y_exact| <= 2^-9 |Y_exact| + 1e-3 rms(Y_exact).
+ * Errors: W8_ERR_NULL, W8_ERR_SHAPE, W8_ERR_ALIGN, W8_ERR_WORKSPACE,
+ *         W8_ERR_ALIAS, W8_ERR_DEVICE, W8_ERR_CUDA.
+ */
+int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
+                 const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* w8_error_string -- static text for a w8_status value. */
+const char *w8_error_string(int status);
+
+/*
+ * w8_device_status -- diagnostic: synchronizes `stream`, then reads and
+ * clears the device status word of the current device into *out.  0 means
+ * no kernel gave up a wait; otherwise bit 0 is set and bits 8..15 name the
+ * wait site.  Returns W8_OK, W8_ERR_NULL or W8_ERR_CUDA.
+ */
+int w8_device_status(void *stream, uint32_t *out);
+
+/*
+ * w8_test_bounded_wait -- self-test of the bounded-wait machinery: launches
+ * one thread that waits on a barrier nothing will complete, with the given
+ * limit in nanoseconds (1e3 .. 5e9); the wait gives up, records site 0xEE in
+ * the device status word and the kernel returns.  Used by the tests to
+ * check that a wait that runs out ends the kernel cleanly.
+ */
+int w8_test_bounded_wait(uint64_t limit_ns, void *stream);
+
+/* w8_version -- ABI version of this header (major * 100 + minor). */
+int w8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W8A16_H */

@@ -1,0 +1,282 @@
+// Decode-regime W8A16 linear (M <= 16 tokens): Y = X . dequant(q) (+ bias).
+//
+// For few tokens the cost is streaming the int8 weight from HBM once
+// (TPU-MLIR ChatGLM2 W8A16 article, section 4: when the left matrix is
+// small, loading the right matrix dominates, int8 halves that load, and the
+// cast and scale hide under it).  Design:
+//  - The packed weight is a sequence of T = ceil(N/128) * ceil(K/64) tiles
+//    of 8 KB, channel-block major.  A single wave of G CTAs (one per SM)
+//    splits that sequence into G equal contiguous ranges (stream-K split),
+//    so every SM streams the same number of bytes and no tail wave exists.
+//  - One producer warp per CTA moves each stage (up to 4 tiles = 32 KB, plus
+//    the matching 64-wide slices of X) into a 4-stage shared-memory ring
+//    with one 1-D bulk copy (cp.async.bulk) and 2-D TMA loads; 8 consumer
+//    warps each own 16 of the tile's 128 channels.
+//  - Consumers widen int8 to fp16 in registers (prmt into the exponent
+//    pattern of 1024, then one fp16x2 subtraction) and accumulate in fp32
+//    with mma.sync m16n8k16 (channels as the MMA rows, tokens as its 8 or
+//    16 columns), so conversion plus multiply-add stay a small fraction of
+//    the issue budget even at 16 tokens.
+//  - A channel block whose K range is split between CTAs is finished by the
+//    last CTA to arrive (an atomic counter per block, reset by that CTA):
+//    it adds the fp32 partials of all contributors in CTA order, so the
+//    result does not depend on arrival order, then applies scale and bias.
+#pragma once
+
+#include "common.cuh"
+
+namespace w8 {
+namespace decode {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kTilesPerStage = 4;
+constexpr int kStages = 4;
+constexpr int kTileBytes = 8192;
+constexpr int kStageW = kTilesPerStage * kTileBytes;
+
+template <int MT>
+struct Cfg {
+    static constexpr int kXRows = 8 * MT;                // token rows per X box
+    static constexpr int kXBoxBytes = kXRows * 128;      // box {64 fp16, kXRows}
+    static constexpr int kStageX = kTilesPerStage * kXBoxBytes;
+    static constexpr int kStageBytes = kStageW + kStageX;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+    static constexpr int kPartialFloats = kConsumerWarps * 4 * MT * 32;   // per slot
+};
+
+// Workspace: [counters: NB int32, padded to 256 B][partials: 2G slots]
+constexpr int kMaxPartialFloats = Cfg<2>::kPartialFloats;
+
+struct Params {
+    const uint8_t *packed;
+    const uint16_t *scales;
+    const uint16_t *bias;   // may be null
+    uint16_t *Y;
+    int *counters;
+    float *partials;
+    int M;
+    int64_t N;
+    int KB;      // ceil(K / 64)
+    int64_t T;   // tiles
+    int G;       // CTAs
+};
+
+__device__ __forceinline__ int64_t range_start(int i, int64_t T, int G) {
+    return (int64_t)i * T / G;
+}
+// CTA whose range holds tile t.
+__device__ __forceinline__ int owner_of(int64_t t, int64_t T, int G) {
+    return (int)(((t + 1) * (int64_t)G - 1) / T);
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint16_t out_f16(float acc, float s, float b) {
+    return __half_as_ushort(__float2half_rn(fmaf(acc, s, b)));
+}
+
+// Thread (g = lane/4, t = lane%4) of consumer warp w holds, for token tile
+// mt, acc[mt] = Y^T[n][m] at n = 16w+g (+8 for elements 2,3) and
+// m = 8mt + 2t (+1 for elements 1,3).
+template <int MT>
+__device__ __forceinline__ void store_y(const Params &p, int64_t b, int warp, int lane,
+                                        const float (&acc)[MT][4]) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int64_t n = b * 128 + 16 * warp + g + 8 * half;
+        if (n >= p.N) continue;
+        const float s = __half2float(__ushort_as_half(p.scales[n]));
+        const float bb = p.bias ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int m = 8 * mt + 2 * t + e;
+                if (m < p.M) p.Y[(int64_t)m * p.N + n] = out_f16(acc[mt][2 * half + e], s, bb);
+            }
+        }
+    }
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
+    using C = Cfg<MT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ uint64_t full[kStages], empty[kStages];
+    __shared__ uint64_t fix_bar;
+    __shared__ int last_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int cta = blockIdx.x;
+    const int64_t t_begin = range_start(cta, p.T, p.G);
+    const int64_t t_end = range_start(cta + 1, p.T, p.G);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        mbar_init(&fix_bar, kConsumerWarps * 32);
+        fence_barrier_init();
+        prefetch_tensormap(&tmap_x);
+    }
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t policy = policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int64_t t = t_begin; t < t_end;) {
+                const int kb = (int)(t % p.KB);
+                const int cnt = (int)min64(kTilesPerStage, min64(t_end - t, p.KB - kb));
+                if (!mbar_wait(&empty[stage], phase ^ 1u, SITE_DEC_EMPTY)) break;
+                uint8_t *ws = base + stage * C::kStageBytes;
+                uint8_t *xs = ws + kStageW;
+                mbar_arrive_expect_tx(&full[stage], cnt * (kTileBytes + C::kXBoxBytes));
+                bulk_g2s_hint(ws, p.packed + t * kTileBytes, cnt * kTileBytes, &full[stage], policy);
+                for (int j = 0; j < cnt; ++j)
+                    tma_load_2d(xs + j * C::kXBoxBytes, &tmap_x, (kb + j) * 64, 0, &full[stage]);
+                t += cnt;
+                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int g = lane >> 2, tq = lane & 3;
+    const int h = (g >> 1) & 3;                     // chunk swizzle of rows 16w+g, 16w+g+8
+    const int row_lo = 16 * warp + g;
+    const int a_off_lo = row_lo * 64 + ((tq ^ h) << 4);
+    const int a_off_hi = (row_lo + 8) * 64 + ((tq ^ h) << 4);
+    int x_off[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int m = 8 * mt + g;
+        x_off[mt][0] = m * 128 + (((2 * tq) ^ (m & 7)) << 4);
+        x_off[mt][1] = m * 128 + (((2 * tq + 1) ^ (m & 7)) << 4);
+    }
+
+    float acc[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][e] = 0.0f;
+
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t fix_phase = 0;
+    const int64_t first_b = t_begin / p.KB;
+    int64_t seg_start = t_begin;
+
+    for (int64_t t = t_begin; t < t_end;) {
+        const int64_t b = t / p.KB;
+        const int kb = (int)(t % p.KB);
+        const int cnt = (int)min64(kTilesPerStage, min64(t_end - t, p.KB - kb));
+        if (!mbar_wait(&full[stage], phase, SITE_DEC_FULL)) return;
+        const uint8_t *ws = base + stage * C::kStageBytes;
+        const uint8_t *xs = ws + kStageW;
+        for (int j = 0; j < cnt; ++j) {
+            const uint8_t *tile = ws + j * kTileBytes;
+            const uint4 alo = *reinterpret_cast<const uint4 *>(tile + a_off_lo);
+            const uint4 ahi = *reinterpret_cast<const uint4 *>(tile + a_off_hi);
+            uint4 xv[MT][2];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                xv[mt][0] = *reinterpret_cast<const uint4 *>(xs + j * C::kXBoxBytes + x_off[mt][0]);
+                xv[mt][1] = *reinterpret_cast<const uint4 *>(xs + j * C::kXBoxBytes + x_off[mt][1]);
+            }
+            const uint32_t wl[4] = {alo.x, alo.y, alo.z, alo.w};
+            const uint32_t wh[4] = {ahi.x, ahi.y, ahi.z, ahi.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint32_t a0 = unbias2(widen_lo2(wl[jj]));   // row g,   k +0,+1
+                const uint32_t a1 = unbias2(widen_lo2(wh[jj]));   // row g+8, k +0,+1
+                const uint32_t a2 = unbias2(widen_hi2(wl[jj]));   // row g,   k +2,+3
+                const uint32_t a3 = unbias2(widen_hi2(wh[jj]));   // row g+8, k +2,+3
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const uint4 &xq = xv[mt][jj >> 1];
+                    const uint32_t b0 = (jj & 1) ? xq.z : xq.x;
+                    const uint32_t b1 = (jj & 1) ? xq.w : xq.y;
+                    mma_16816(acc[mt], a0, a1, a2, a3, b0, b1);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        t += cnt;
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+
+        if (t == t_end || t % p.KB == 0) {
+            // segment [seg_start, t) of channel block b is complete
+            const bool whole = (seg_start % p.KB == 0) && (t - seg_start == p.KB);
+            if (whole) {
+                store_y<MT>(p, b, warp, lane, acc);
+            } else {
+                const int slot = (b == first_b) ? 2 * cta : 2 * cta + 1;
+                float *mine = p.partials + (int64_t)slot * C::kPartialFloats;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        mine[(warp * 4 * MT + 4 * mt + e) * 32 + lane] = acc[mt][e];
+                __threadfence();
+                mbar_arrive(&fix_bar);
+                if (!mbar_wait(&fix_bar, fix_phase, SITE_DEC_FULL)) return;
+                fix_phase ^= 1u;
+                const int j_first = owner_of(b * p.KB, p.T, p.G);
+                const int j_last = owner_of((b + 1) * p.KB - 1, p.T, p.G);
+                if (threadIdx.x == 0) {
+                    const int old = atomicAdd(&p.counters[b], 1);
+                    last_flag = (old == j_last - j_first);
+                }
+                mbar_arrive(&fix_bar);
+                if (!mbar_wait(&fix_bar, fix_phase, SITE_DEC_FULL)) return;
+                fix_phase ^= 1u;
+                if (last_flag) {
+                    __threadfence();
+                    float sum[MT][4];
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sum[mt][e] = 0.0f;
+                    for (int j = j_first; j <= j_last; ++j) {
+                        const int sj = (range_start(j, p.T, p.G) / p.KB == b) ? 2 * j : 2 * j + 1;
+                        const float *src = p.partials + (int64_t)sj * C::kPartialFloats;
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                sum[mt][e] += __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
+                    }
+                    store_y<MT>(p, b, warp, lane, sum);
+                    if (threadIdx.x == 0) p.counters[b] = 0;
+                }
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[mt][e] = 0.0f;
+            seg_start = t;
+        }
+    }
+}
+
+}  // namespace decode
+}  // namespace w8

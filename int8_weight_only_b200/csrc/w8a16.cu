@@ -1,0 +1,371 @@
+// libw8a16.so: the C ABI declared in include/w8a16.h.  Host code only
+// validates arguments, builds TMA tensor maps and launches the kernels in
+// quantize.cuh, prepack.cuh, decode.cuh and prefill.cuh on the caller's
+// stream.  Nothing here allocates device memory or synchronizes (except the
+// w8_device_status diagnostic).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <climits>
+#include <mutex>
+
+#include "../../include/w8a16.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "prepack.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+using namespace w8;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int status = W8_OK;   // W8_ERR_DEVICE if not sm_100
+    int sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+// Per-device one-time setup: architecture check, SM count, kernel attributes.
+int device_info(DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W8_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return W8_ERR_CUDA;
+        d.sms = sms;
+        d.status = (major == 10 && minor == 0) ? W8_OK : W8_ERR_DEVICE;
+        if (d.status == W8_OK) {
+            cudaError_t e = cudaSuccess;
+            e = cudaFuncSetAttribute(decode::decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     decode::Cfg<1>::kSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(decode::decode_kernel<2>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         decode::Cfg<2>::kSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(prefill::prefill_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         prefill::kSmemBytes);
+            const int qmax = 201 * 1024;
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(quant::quantize_kernel<float, 32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, qmax);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(quant::quantize_kernel<float, 16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, qmax);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(quant::quantize_kernel<__half, 32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, qmax);
+            if (e != cudaSuccess) return W8_ERR_CUDA;
+        }
+        d.ready = true;
+    }
+    *out = &d;
+    return d.status;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem`-byte elements.
+int make_map_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType dtype, int elem, uint64_t cols,
+                uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return W8_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)elem};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W8_OK : W8_ERR_CUDA;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool overlap(const void *a, size_t an, const void *b, size_t bn) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return an && bn && x < y + bn && y < x + an;
+}
+
+inline int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? W8_OK : W8_ERR_CUDA;
+}
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- quantize
+template <typename T, int BN>
+int launch_quantize(const void *W, CUtensorMapDataType dt, int64_t K, int64_t N, int8_t *q,
+                    uint16_t *scales, cudaStream_t st) {
+    constexpr int elem = sizeof(T);
+    constexpr int box_bytes = quant::kBoxRows * BN * elem;
+    constexpr int64_t target_rows = (64 * 1024) / (BN * elem);   // ~64 KB per CTA
+    constexpr int64_t resident_max = (200 * 1024) / box_bytes;  // boxes
+    int cq = (int)std::min<int64_t>(8, std::max<int64_t>(1, cdiv(K, target_rows)));
+    int64_t kc = cdiv(cdiv(K, cq), quant::kBoxRows) * quant::kBoxRows;
+    int64_t nbox = kc / quant::kBoxRows;
+    int nbuf = (int)std::min<int64_t>({nbox, resident_max, (int64_t)quant::kMaxBoxes});
+    if (nbox > nbuf) nbuf = (int)std::min<int64_t>(8, nbuf);   // streaming: 8 boxes in flight
+    if (kc > INT32_MAX) return W8_ERR_SHAPE;
+
+    CUtensorMap map;
+    int rc = make_map_2d(&map, W, dt, elem, (uint64_t)N, (uint64_t)K, BN, quant::kBoxRows,
+                         CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc != W8_OK) return rc;
+
+    const int64_t strips = cdiv(N, BN);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(strips * cq), 1, 1);
+    cfg.blockDim = dim3(quant::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)nbuf * box_bytes + 1024;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cq;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T, BN>, map, K, N, (int)kc, nbuf, q, scales) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return W8_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int w8_version(void) { return 100; }
+
+const char *w8_error_string(int status) {
+    switch (status) {
+        case W8_OK: return "ok";
+        case W8_ERR_NULL: return "a required pointer is NULL";
+        case W8_ERR_SHAPE: return "a size is out of range or not a multiple of 8";
+        case W8_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+        case W8_ERR_DTYPE: return "unknown weight dtype";
+        case W8_ERR_WORKSPACE: return "workspace missing or too small";
+        case W8_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
+        case W8_ERR_TIMEOUT: return "a bounded device wait ran out";
+        case W8_ERR_ALIAS: return "output overlaps an input";
+        case W8_ERR_DEVICE: return "current device is not sm_100 (B200)";
+        default: return "unknown status";
+    }
+}
+
+int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
+                            uint16_t *scales, void *stream) {
+    if (!W || !q || !scales) return W8_ERR_NULL;
+    if (w_dtype != W8_F32 && w_dtype != W8_F16) return W8_ERR_DTYPE;
+    if (K < 1 || N < 0 || N % 8 != 0 || K > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX * 8)
+        return W8_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(q) || !aligned16(scales)) return W8_ERR_ALIGN;
+    const size_t welem = w_dtype == W8_F32 ? 4 : 2;
+    if (overlap(W, (size_t)K * N * welem, q, (size_t)K * N) ||
+        overlap(W, (size_t)K * N * welem, scales, (size_t)N * 2) ||
+        overlap(q, (size_t)K * N, scales, (size_t)N * 2))
+        return W8_ERR_ALIAS;
+    if (N == 0) return W8_OK;
+    DeviceInfo *d = nullptr;
+    int rc = device_info(&d);
+    if (rc != W8_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (w_dtype == W8_F32) {
+        // keep each CTA's strip resident in shared memory: 32 columns while
+        // it fits the cluster, else 16 (64-byte rows), else stream twice
+        const int64_t per_cta32 = cdiv(cdiv(K, 8), 64) * 64 * 32 * 4;
+        if (per_cta32 <= 112 * 1024 || cdiv(cdiv(K, 8), 64) * 64 * 16 * 4 > 200 * 1024)
+            return launch_quantize<float, 32>(W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, st);
+        return launch_quantize<float, 16>(W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, st);
+    }
+    return launch_quantize<__half, 32>(W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, st);
+}
+
+size_t w8_prepacked_bytes(int64_t K, int64_t N) {
+    if (K < 1 || N < 1) return 0;
+    return (size_t)cdiv(N, W8_TILE_N) * (size_t)cdiv(K, W8_TILE_K) * W8_TILE_BYTES;
+}
+
+static int pack_args(const void *a, const void *b, int64_t K, int64_t N) {
+    if (!a || !b) return W8_ERR_NULL;
+    if (K < 1 || N < 1 || N % 8 != 0 || cdiv(K, 64) > 65535 * 1024LL || cdiv(N, 128) > 65535)
+        return W8_ERR_SHAPE;
+    if (!aligned16(a) || !aligned16(b)) return W8_ERR_ALIGN;
+    if (overlap(a, w8_prepacked_bytes(K, N), b, w8_prepacked_bytes(K, N))) return W8_ERR_ALIAS;
+    return W8_OK;
+}
+
+int w8_prepack(const int8_t *q, int64_t K, int64_t N, uint8_t *packed, void *stream) {
+    int rc = pack_args(q, packed, K, N);
+    if (rc != W8_OK) return rc;
+    DeviceInfo *d = nullptr;
+    if ((rc = device_info(&d)) != W8_OK) return rc;
+    const int KB = (int)cdiv(K, 64);
+    dim3 grid((unsigned)KB, (unsigned)cdiv(N, 128));
+    pack::prepack_kernel<<<grid, pack::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(q, K, N, KB,
+                                                                                        packed);
+    return launch_status();
+}
+
+int w8_unpack(const uint8_t *packed, int64_t K, int64_t N, int8_t *q, void *stream) {
+    int rc = pack_args(packed, q, K, N);
+    if (rc != W8_OK) return rc;
+    DeviceInfo *d = nullptr;
+    if ((rc = device_info(&d)) != W8_OK) return rc;
+    const int KB = (int)cdiv(K, 64);
+    dim3 grid((unsigned)KB, (unsigned)cdiv(N, 128));
+    pack::unpack_kernel<<<grid, pack::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(packed, K, N, KB,
+                                                                                       q);
+    return launch_status();
+}
+
+// Decode split: one CTA per SM (never more CTAs than tiles).
+static int decode_grid(int sms, int64_t T) { return (int)std::max<int64_t>(1, std::min<int64_t>(T, sms)); }
+
+static size_t decode_workspace(int sms, int64_t K, int64_t N) {
+    const int64_t NB = cdiv(N, 128), T = NB * cdiv(K, 64);
+    const int G = decode_grid(sms, T);
+    const size_t counters = (size_t)cdiv(NB * 4, 256) * 256;
+    const size_t partials = (size_t)2 * G * decode::kMaxPartialFloats * sizeof(float);
+    return counters + partials;
+}
+
+size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+    if (M < 1 || M > 16 || K < 1 || N < 1) return 0;
+    DeviceInfo *d = nullptr;
+    if (device_info(&d) != W8_OK) return 0;
+    return decode_workspace(d->sms, K, N);
+}
+
+int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
+                 const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
+                 void *workspace, size_t workspace_bytes, void *stream) {
+    if (!X || !packed || !scales || !Y) return W8_ERR_NULL;
+    if (M < 0 || K < 1 || N < 1 || K % 8 != 0 || N % 8 != 0 || M > (int64_t)INT32_MAX ||
+        K > (int64_t)INT32_MAX || cdiv(K, 64) > INT32_MAX)
+        return W8_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(Y) ||
+        (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
+        return W8_ERR_ALIGN;
+    const size_t ybytes = (size_t)M * N * 2;
+    if (overlap(Y, ybytes, X, (size_t)M * K * 2) ||
+        overlap(Y, ybytes, packed, w8_prepacked_bytes(K, N)) ||
+        overlap(Y, ybytes, scales, (size_t)N * 2) || (bias && overlap(Y, ybytes, bias, (size_t)N * 2)))
+        return W8_ERR_ALIAS;
+    if (M == 0) return W8_OK;
+    DeviceInfo *d = nullptr;
+    int rc = device_info(&d);
+    if (rc != W8_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int KB = (int)cdiv(K, 64);
+    const int64_t NB = cdiv(N, 128);
+
+    if (M <= 16) {
+        const size_t need = decode_workspace(d->sms, K, N);
+        if (!workspace || workspace_bytes < need) return W8_ERR_WORKSPACE;
+        if (overlap(workspace, need, Y, ybytes) || overlap(workspace, need, X, (size_t)M * K * 2))
+            return W8_ERR_ALIAS;
+        const int MT = M <= 8 ? 1 : 2;
+        CUtensorMap map;
+        rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
+                         8 * MT, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc != W8_OK) return rc;
+        decode::Params p;
+        p.packed = packed;
+        p.scales = scales;
+        p.bias = bias;
+        p.Y = Y;
+        p.counters = static_cast<int *>(workspace);
+        p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                               (size_t)cdiv(NB * 4, 256) * 256);
+        p.M = (int)M;
+        p.N = N;
+        p.KB = KB;
+        p.T = NB * KB;
+        p.G = decode_grid(d->sms, p.T);
+        if (MT == 1)
+            decode::decode_kernel<1><<<p.G, decode::kThreads, decode::Cfg<1>::kSmemBytes, st>>>(map, p);
+        else
+            decode::decode_kernel<2><<<p.G, decode::kThreads, decode::Cfg<2>::kSmemBytes, st>>>(map, p);
+        return launch_status();
+    }
+
+    CUtensorMap map;
+    rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
+                     prefill::kBT, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != W8_OK) return rc;
+    prefill::Params p;
+    p.packed = packed;
+    p.scales = scales;
+    p.bias = bias;
+    p.Y = Y;
+    p.M = (int)M;
+    p.N = N;
+    p.KB = KB;
+    p.TT = (int)cdiv(M, prefill::kBT);
+    p.tiles = NB * p.TT;
+    const int grid = (int)std::min<int64_t>(p.tiles, d->sms);
+    prefill::prefill_kernel<<<grid, prefill::kThreads, prefill::kSmemBytes, st>>>(map, p);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------- diagnostics
+namespace {
+__global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        // nothing ever arrives on `bar`: the wait must give up by itself
+        mbar_wait(&bar, 0, SITE_SELFTEST, limit_ns);
+    }
+}
+}  // namespace
+
+int w8_test_bounded_wait(uint64_t limit_ns, void *stream) {
+    if (limit_ns < 1000 || limit_ns > 5000000000ull) return W8_ERR_SHAPE;
+    DeviceInfo *d = nullptr;
+    int rc = device_info(&d);
+    if (rc != W8_OK) return rc;
+    bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    return launch_status();
+}
+
+int w8_device_status(void *stream, uint32_t *out) {
+    if (!out) return W8_ERR_NULL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned int v = 0, zero = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return W8_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return W8_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return W8_ERR_CUDA;
+    *out = v;
+    return W8_OK;
+}
+
+}  // extern "C"

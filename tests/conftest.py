@@ -28,3 +28,12 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def w8lib():
+    """The product library, built in-tree if missing (no GPU needed)."""
+    from int8_weight_only_b200 import build as _build
+    import int8_weight_only_b200 as w8
+    _build.build()
+    return w8.load_library()

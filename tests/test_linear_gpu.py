@@ -1,0 +1,198 @@
+"""GPU W8A16 linear against the oracle.
+
+Every case runs the product pipeline on the GPU (quantize -> prepack ->
+linear) and the oracle on the same host inputs (its own quantize -> fp64
+linear).  Y must satisfy |Y - Y_ref| <= 2^-9 |Y_ref| + 1e-3 rms(Y_ref)
+element-wise; where the arithmetic is exact, bit equality is required.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+from tests.gpu_helpers import SEED, assert_close, gpu_pipeline, to_gpu, to_np, w8
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(M, K, N, tid, bias=True, outliers=0.001):
+    W = synthetic.weights(K, N, SEED, tid, outlier_frac=outliers)
+    X = synthetic.activations(M, K, SEED, tid + 1)
+    b = synthetic.bias(N, SEED, tid + 2) if bias else None
+    return W, X, b
+
+
+def _check_full(M, K, N, tid, bias=True):
+    W, X, b = _case(M, K, N, tid, bias)
+    qg, sg, Yg = gpu_pipeline(W, X, b)
+    qo, so = oracle.quantize(W)
+    assert np.array_equal(qg, qo) and np.array_equal(sg.view(np.uint16), so.view(np.uint16))
+    Yref = oracle.linear(X, qo, so, b)
+    return assert_close(Yg, Yref, f"M={M} K={K} N={N}")
+
+
+# ---------------------------------------------------------------- decode (M <= 16)
+DECODE_SHAPES = [(256, 512), (64, 8), (200, 136), (1024, 1032), (4096, 4608), (13696, 264)]
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
+@pytest.mark.parametrize("K,N", DECODE_SHAPES)
+def test_decode_matches_oracle(M, K, N):
+    _check_full(M, K, N, 2000 + K + N + M, bias=(M % 2 == 1))
+
+
+# ---------------------------------------------------------------- prefill (M > 16)
+PREFILL_SHAPES = [(256, 512), (64, 136), (520, 264), (4096, 384)]
+
+
+@pytest.mark.parametrize("M", [17, 64, 128, 129, 300])
+@pytest.mark.parametrize("K,N", PREFILL_SHAPES)
+def test_prefill_matches_oracle(M, K, N):
+    _check_full(M, K, N, 3000 + K + N + M, bias=(M % 2 == 0))
+
+
+def test_tiny_workload_both_paths():
+    # 4 x 256 activations, 256 x 512 weight (the smallest workload), then the
+    # same weight through the tensor-core path with 4 copies of X stacked
+    _check_full(4, 256, 512, synthetic.tensor_id(1, 0, 0, 0), bias=False)
+    W, X, _ = _case(4, 256, 512, synthetic.tensor_id(1, 0, 0, 0), bias=False)
+    X32 = np.concatenate([X] * 8, axis=0)
+    qg, sg, Yg = gpu_pipeline(W, X32)
+    qo, so = oracle.quantize(W)
+    assert_close(Yg, oracle.linear(X32, qo, so), "stacked")
+
+
+# ---------------------------------------------------------------- exact cases
+@pytest.mark.parametrize("M", [1, 5, 16, 40, 200])
+def test_exact_integer_inputs_bit_exact(M):
+    # integer X and power-of-two-multiple weights: every product and partial
+    # sum is exact in fp32, so Y must equal the exact value rounded to fp16
+    rng = np.random.default_rng(M)
+    K, N = 512, 264
+    X = rng.integers(-8, 9, size=(M, K)).astype(np.float16)
+    s0 = 2.0 ** rng.integers(-10, -4, size=N)
+    j = rng.integers(-127, 128, size=(K, N))
+    j[0] = 127
+    W = (j * s0).astype(np.float32)
+    b = (rng.integers(-64, 64, size=N) / 16.0).astype(np.float16)
+    qg, sg, Yg = gpu_pipeline(W, X, b)
+    qo, so = oracle.quantize(W)
+    Yref = oracle.linear(X, qo, so, b)
+    assert np.array_equal(Yg.view(np.uint16), Yref.astype(np.float16).view(np.uint16))
+
+
+def test_unit_rows_select_weight_rows():
+    K, N = 320, 136
+    W, _, _ = _case(1, K, N, 3500, bias=False)
+    ks = [0, 63, 64, 319]
+    for M in (len(ks), 32):
+        X = np.zeros((M, K), dtype=np.float16)
+        for m in range(M):
+            X[m, ks[m % len(ks)]] = 1.0
+        qg, sg, Yg = gpu_pipeline(W, X)
+        qo, so = oracle.quantize(W)
+        Yref = oracle.linear(X, qo, so)
+        assert np.array_equal(Yg.view(np.uint16), Yref.astype(np.float16).view(np.uint16))
+
+
+def test_deterministic_across_calls():
+    m = w8()
+    for M in (1, 16, 100):
+        W, X, b = _case(M, 2048, 1024, 3600 + M)
+        q, s = m.quantize(to_gpu(W))
+        packed = m.prepack(q)
+        Xg, bg = to_gpu(X), to_gpu(b)
+        Y1 = to_np(m.linear(Xg, packed, s, bg))
+        Y2 = to_np(m.linear(Xg, packed, s, bg))
+        assert np.array_equal(Y1.view(np.uint16), Y2.view(np.uint16))
+
+
+def test_workspace_reused_across_shapes():
+    # the split-K counters are reset by each call, so one workspace serves
+    # calls of different shapes back to back
+    for (M, K, N) in [(1, 4096, 512), (3, 64, 8), (16, 1000, 1032), (1, 4096, 512)]:
+        _check_full(M, K, N, 3700 + K + N)
+
+
+def test_workspace_too_small_is_rejected():
+    torch = pytest.importorskip("torch")
+    m = w8()
+    W, X, _ = _case(1, 256, 512, 3800)
+    q, s = m.quantize(to_gpu(W))
+    packed = m.prepack(q)
+    need = m.workspace_bytes(1, 256, 512)
+    assert need > 0
+    ws = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(m.W8Error) as e:
+        m.linear(to_gpu(X), packed, s, workspace=ws)
+    assert e.value.status == -5
+    assert m.workspace_bytes(17, 256, 512) == 0
+
+
+def test_empty_batch():
+    torch = pytest.importorskip("torch")
+    m = w8()
+    W, _, _ = _case(1, 64, 128, 3900)
+    q, s = m.quantize(to_gpu(W))
+    packed = m.prepack(q)
+    Y = m.linear(torch.zeros((0, 64), dtype=torch.float16, device="cuda"), packed, s)
+    assert tuple(Y.shape) == (0, 128)
+
+
+# ---------------------------------------------------------------- full-size workloads
+def test_chatglm2_h_to_4h_decode_full():
+    # M = 1, 4096 x 27392, 0.1 % outliers: every output checked
+    tid = synthetic.tensor_id(2, 0, 0, 0)
+    K, N = 4096, 27392
+    W = synthetic.weights(K, N, SEED, tid, outlier_frac=0.001)
+    X = synthetic.activations(1, K, SEED, tid + 1)
+    qg, sg, Yg = gpu_pipeline(W, X)
+    rng = np.random.default_rng(11)
+    cols = np.sort(rng.choice(N, 1024, replace=False))
+    qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
+    assert np.array_equal(qg[:, cols], qo)
+    # the oracle's fp64 product over all channels, with the oracle's codes
+    # for the sampled channels and the same codes elsewhere checked above
+    Yref = oracle.linear(X, qo, so)
+    assert_close(Yg[:, cols], Yref, "h-to-4h decode sample")
+    qall, sall = oracle.quantize(W)
+    assert_close(Yg, oracle.linear(X, qall, sall), "h-to-4h decode all")
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+def test_chatglm2_decode_layer_sampled(M):
+    rng = np.random.default_rng(M)
+    for i, (K, N) in enumerate(synthetic.WORKLOADS["chatglm2_decode_set"]["matrices"]):
+        tid = synthetic.tensor_id(3, 0, i, 0)
+        W = synthetic.weights(K, N, SEED, tid, outlier_frac=0.001)
+        X = synthetic.activations(M, K, SEED, synthetic.tensor_id(3, M, i, 1))
+        _, _, Yg = gpu_pipeline(W, X)
+        cols = np.sort(rng.choice(N, 256, replace=False))
+        qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
+        assert_close(Yg[:, cols], oracle.linear(X, qo, so), f"layer matrix {i} M={M}")
+
+
+@pytest.mark.parametrize("M", [512, 1024, 2048])
+def test_chatglm2_prefill_sampled(M):
+    rng = np.random.default_rng(M)
+    for i, (K, N) in enumerate(synthetic.WORKLOADS["chatglm2_prefill"]["matrices"]):
+        tid = synthetic.tensor_id(4, 0, i, 0)
+        W = synthetic.weights(K, N, SEED, tid, outlier_frac=0.001)
+        X = synthetic.activations(M, K, SEED, synthetic.tensor_id(4, M, i, 1))
+        _, _, Yg = gpu_pipeline(W, X)
+        cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 62, replace=False)]))
+        qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
+        assert_close(Yg[:, cols], oracle.linear(X, qo, so), f"prefill matrix {i} M={M}")
+
+
+def test_bert_base_4096_tokens_sampled():
+    rng = np.random.default_rng(5)
+    for i, (K, N) in enumerate(synthetic.WORKLOADS["bert_base_4096_tokens"]["matrices"]):
+        tid = synthetic.tensor_id(5, 0, i, 0)
+        W = synthetic.weights(K, N, SEED, tid)
+        X = synthetic.activations(4096, K, SEED, tid + 1)
+        b = synthetic.bias(N, SEED, tid + 2)
+        _, _, Yg = gpu_pipeline(W, X, b)
+        cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 62, replace=False)]))
+        qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
+        assert_close(Yg[:, cols], oracle.linear(X, qo, so, b[cols]), f"bert matrix {i}")

@@ -1,0 +1,91 @@
+"""GPU quantization is bit-exact with the oracle (q and scales), on ragged
+shapes, both weight dtypes, the edge columns the method has, and every
+internal path (resident strip, 16-column strip, two-pass streaming)."""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+from tests.gpu_helpers import SEED, to_gpu, to_np, w8
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(256, 512), (1, 8), (7, 24), (63, 136), (65, 264), (200, 40), (1000, 1032), (4096, 512)]
+
+
+def _gpu_quant(W):
+    q, s = w8().quantize(to_gpu(W))
+    return to_np(q), to_np(s)
+
+
+def _check(W):
+    qo, so = oracle.quantize(W)
+    qg, sg = _gpu_quant(W)
+    assert np.array_equal(sg.view(np.uint16), so.view(np.uint16))
+    assert np.array_equal(qg, qo)
+
+
+@pytest.mark.parametrize("dtype", [np.float32, np.float16])
+@pytest.mark.parametrize("K,N", SHAPES)
+def test_quantize_bit_exact(K, N, dtype):
+    W = synthetic.weights(K, N, SEED, 1000 + K + N, outlier_frac=0.001).astype(dtype)
+    _check(W)
+
+
+def test_quantize_edge_columns():
+    K, N = 300, 64
+    W = synthetic.weights(K, N, SEED, 1100)
+    W[:, 0] = 0.0                                           # all-zero column
+    W[:, 1] = -0.0
+    W[:, 2] = np.float32(2.0 ** -24) * np.arange(K) / K     # subnormal fp16 scale
+    W[:5, 3] = np.float32(127 * 1.4 * 2.0 ** -24)           # clip engages
+    W[5:, 3] = 0.0
+    s0 = float(np.float16(0.0123))
+    j = (np.arange(K) % 255) - 127
+    W[:, 4] = (j * s0).astype(np.float32)                   # exact multiples
+    W[:, 5] = np.concatenate([[127 * s0], (np.arange(K - 1) % 200 - 100 + 0.5) * s0])  # ties
+    W[:, 6] = 1e-30                                         # fp32 subnormal -> zero scale
+    W[7, 7] = 3.0e4                                         # one large outlier
+    _check(W)
+
+
+def test_quantize_16_column_strip_path():
+    # K = 13696 (the ChatGLM2 4h-to-h input width) in fp32 uses 16-column strips
+    W = synthetic.weights(13696, 256, SEED, 1200, outlier_frac=0.001)
+    _check(W)
+
+
+def test_quantize_streaming_path():
+    # a strip too tall to stay in cluster shared memory is read twice
+    W = synthetic.weights(30000, 72, SEED, 1300, outlier_frac=0.001)
+    _check(W)
+
+
+def test_quantize_repeatable():
+    W = synthetic.weights(512, 264, SEED, 1400)
+    a = _gpu_quant(W)
+    b = _gpu_quant(W)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_quantize_chatglm2_h_to_4h_full_size():
+    # 4096 x 27392 with 0.1 % outliers: all columns against the invariants,
+    # 640 sampled columns (including both ragged ends) bit-exact
+    K, N = 4096, 27392
+    W = synthetic.weights(K, N, SEED, synthetic.tensor_id(2, 0, 0, 0), outlier_frac=0.001)
+    qg, sg = _gpu_quant(W)
+    rng = np.random.default_rng(3)
+    cols = np.unique(np.concatenate([np.arange(32), np.arange(N - 32, N),
+                                     rng.choice(N, 576, replace=False)]))
+    qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
+    assert np.array_equal(sg[cols].view(np.uint16), so.view(np.uint16))
+    assert np.array_equal(qg[:, cols], qo)
+    assert qg.min() >= -127 and qg.max() <= 127
+    arg = np.argmax(np.abs(W), axis=0)
+    assert np.all(np.abs(qg[arg, np.arange(N)]) == 127)
+
+
+def test_quantize_bert_base_all_weights():
+    for i, (K, N) in enumerate(synthetic.WORKLOADS["bert_base_4096_tokens"]["matrices"]):
+        W = synthetic.weights(K, N, SEED, synthetic.tensor_id(5, 0, i, 0))
+        _check(W)
