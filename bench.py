@@ -1,0 +1,455 @@
+#!/usr/bin/env python3
+"""Benchmark of the W8A16 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Headline metric: weight GB/s of the decode linear at M = 1 on the
+ChatGLM2-6B h-to-4h shape (X fp16 [1, 4096] . W int8 [4096, 27392]).  One
+step is one w8a16_linear call; each step reads a different copy of the
+packed weight (6 copies, 673 MB > 126 MB L2), so no step is served from L2.
+The timed region replays a CUDA graph of those calls; it is bracketed by a
+barrier and a device synchronize and timed with CUDA events on the launching
+stream, max over ranks.  The same JSON line also reports, measured in the
+same run:
+  - prefill: TFLOP/s of the M = 2048 linear on the same weight (two weight
+    copies alternate; X 16 MB);
+  - quantize / prepack: the one-time weight conversion (fp32 W 449 MB ->
+    int8 q + fp16 scales; q -> packed tiles);
+  - e2e: the decode metric with the per-step H2D copy of X from pinned host
+    memory and the D2H copy of Y inside the timed region;
+  - roofline of the dominant kernel, clocks sampled during the timed region,
+    and the CPU oracle timed on a bounded sample (rank 0).
+
+N > 1: every rank runs the same independent workload on its own GPU (the
+problems are independent; there is no data-path collective), value = units
+of all ranks / max-over-ranks time ("weak" scaling).
+
+--impl reference times the CPU oracle (plain C, one thread) on the same
+metric and workload, each step a bounded column slab of the weight.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W8A16 GEMM weight GB/s (M=1, 4096×27392) and TFLOP/s (M=2048) on 1 B200"
+K_DIM, N_DIM, M_DECODE, M_PREFILL = 4096, 27392, 1, 2048
+N_COPIES = 6                  # 6 x 112 MB rotating weight copies > 4 x L2
+WORKLOAD = ("chatglm2_h_to_4h_decode: X fp16 [1,4096] . W int8 [4096,27392] "
+            "(per-channel int8, fp16 scales), W ~ N(0,0.02) with 0.1% N(0,0.2) outliers")
+FALLBACK_HBM, FALLBACK_TF = 6650.0, 1590.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return FALLBACK_HBM, FALLBACK_TF, 1400.0, "fallback"
+
+
+def kernel_source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "int8_weight_only_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, sources):
+    """DRAM bytes per launch from a committed ncu summary, only if the
+    kernel sources are unchanged since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)[kernel]
+        if t["source_hash"] == kernel_source_hash(sources):
+            return float(t["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap,power.draw")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        self.windows = []
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except Exception:
+                self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = []
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                frac = float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                rows.append((ts + frac, float(parts[1]), float(parts[2]), parts[3:7]))
+            except Exception:
+                continue
+        os.unlink(self.f.name)
+        inside = [r for r in rows if any(a - 0.15 <= r[0] <= b + 0.15 for a, b in self.windows)]
+        use = inside if len(inside) >= 2 else rows
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use),
+                "window": "timed regions" if use is inside else "whole run"}
+
+
+# ------------------------------------------------------------------ helpers
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl" if os.environ.get("W8_BENCH_BACKEND", "nccl") == "nccl" else "gloo",
+                                timeout=datetime.timedelta(seconds=120))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, value: float, device) -> float:
+    if ws == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_replays(graph, n_replays, stream, ws, device, sampler):
+    """Replay `graph` n_replays times between synchronizes; device time in s."""
+    import torch
+    barrier(ws)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(n_replays):
+            graph.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark(t0, time.time())
+    elapsed = start.elapsed_time(end) / 1e3
+    barrier(ws)
+    return max_over_ranks(ws, elapsed, device)
+
+
+def capture(fn, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+# ------------------------------------------------------------------ native arm
+def run_native(args, ws, rank, local):
+    import torch
+    import synthetic
+    import int8_weight_only_b200 as w8
+    from int8_weight_only_b200 import build as w8build
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if rank == 0:
+        w8build.build()
+    barrier(ws)
+    w8.load_library()
+    hbm_peak, tf_peak, tf_sustained, peak_src = peaks()
+    sampler = ClockSampler(local)
+    stream = torch.cuda.Stream(device)
+
+    # ---- inputs (host, seeded) -> device
+    seed = synthetic.SEED + rank
+    tid = synthetic.tensor_id(2, 0, 0, 0)
+    W_host = synthetic.weights(K_DIM, N_DIM, seed, tid, outlier_frac=0.001)
+    X1_host = synthetic.activations(M_DECODE, K_DIM, seed, tid + 1)
+    Xp_host = synthetic.activations(M_PREFILL, K_DIM, seed, synthetic.tensor_id(4, M_PREFILL, 0, 1))
+    W = torch.from_numpy(W_host).to(device)
+    X1 = torch.from_numpy(X1_host).to(device)
+    Xp = torch.from_numpy(Xp_host).to(device)
+    del W_host
+
+    with torch.cuda.stream(stream):
+        q, scales = w8.quantize(W)
+        packed0 = w8.prepack(q)
+        copies = [packed0] + [packed0.clone() for _ in range(N_COPIES - 1)]
+        Y1 = torch.empty((M_DECODE, N_DIM), dtype=torch.float16, device=device)
+        Yp = torch.empty((M_PREFILL, N_DIM), dtype=torch.float16, device=device)
+        ws_need = w8.workspace_bytes(M_DECODE, K_DIM, N_DIM, device)
+        work = torch.zeros((max(ws_need, 1),), dtype=torch.uint8, device=device)
+        # warm-up of every entry point outside capture (one-time device setup)
+        w8.linear(X1, copies[0], scales, out=Y1, workspace=work)
+        w8.linear(Xp, copies[0], scales, out=Yp)
+    torch.cuda.synchronize()
+
+    steps, warmup = args.steps, args.warmup
+
+    # ---- decode (headline): a graph of N_COPIES calls, rotating the weight copy
+    def decode_round():
+        for c in copies:
+            w8.linear(X1, c, scales, out=Y1, workspace=work)
+
+    g_dec = capture(decode_round, stream)
+    n_rep = -(-steps // N_COPIES)
+    steps_done = n_rep * N_COPIES
+    for _ in range(max(1, -(-warmup // N_COPIES))):
+        with torch.cuda.stream(stream):
+            g_dec.replay()
+    torch.cuda.synchronize()
+    t_dec = timed_replays(g_dec, n_rep, stream, ws, device, sampler)
+    dec_s = t_dec / steps_done
+    weight_bytes = K_DIM * N_DIM
+    alg_bytes = weight_bytes + 2 * N_DIM + 2 * M_DECODE * K_DIM + 2 * M_DECODE * N_DIM
+    value = ws * weight_bytes * steps_done / t_dec / 1e9
+    dec_achieved = alg_bytes / dec_s / 1e9
+
+    # ---- prefill M = 2048 (two weight copies alternate: 224 MB > L2)
+    def prefill_round():
+        for c in copies[:2]:
+            w8.linear(Xp, c, scales, out=Yp)
+
+    g_pf = capture(prefill_round, stream)
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            g_pf.replay()
+    torch.cuda.synchronize()
+    n_pf = max(5, args.prefill_reps)
+    t_pf = timed_replays(g_pf, n_pf, stream, ws, device, sampler)
+    pf_s = t_pf / (2 * n_pf)
+    pf_flops = 2.0 * M_PREFILL * K_DIM * N_DIM
+    pf_tflops = pf_flops / pf_s / 1e12
+
+    # ---- quantize (fp32 W 449 MB > L2) and prepack (one-time weight path)
+    q2 = torch.empty_like(q)
+    s2 = torch.empty_like(scales)
+    g_q = capture(lambda: w8.quantize(W, q=q2, scales=s2), stream)
+    g_pk = capture(lambda: w8.prepack(q2, out=copies[1]), stream)
+    for g in (g_q, g_pk):
+        for _ in range(3):
+            with torch.cuda.stream(stream):
+                g.replay()
+    torch.cuda.synchronize()
+    n_q = max(5, args.prefill_reps)
+    t_q = timed_replays(g_q, n_q, stream, ws, device, sampler) / n_q
+    t_pk = timed_replays(g_pk, n_q, stream, ws, device, sampler) / n_q
+    q_bytes = K_DIM * N_DIM * (4 + 1) + 2 * N_DIM
+    pk_bytes = 2 * K_DIM * N_DIM
+    same = bool(torch.equal(q, q2) and torch.equal(scales, s2))
+
+    # ---- e2e: pinned host X -> device, linear, device -> pinned host Y
+    Xh = torch.from_numpy(X1_host).pin_memory()
+    Yh = torch.empty((M_DECODE, N_DIM), dtype=torch.float16).pin_memory()
+    Xd = torch.empty_like(X1)
+
+    def e2e_round():
+        for c in copies:
+            Xd.copy_(Xh, non_blocking=True)
+            w8.linear(Xd, c, scales, out=Y1, workspace=work)
+            Yh.copy_(Y1, non_blocking=True)
+
+    g_e2e = capture(e2e_round, stream)
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            g_e2e.replay()
+    torch.cuda.synchronize()
+    t_e2e = timed_replays(g_e2e, n_rep, stream, ws, device, sampler)
+    e2e_value = ws * weight_bytes * steps_done / t_e2e / 1e9
+
+    clocks = sampler.stop()
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": steps_done,
+        "warmup": warmup,
+        "ms_per_step": round(dec_s * 1e3, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD,
+            "M": M_DECODE, "K": K_DIM, "N": N_DIM,
+            "weights": "int8 per-output-channel, fp16 scales, prepacked tiles",
+            "l2": f"inputs larger than L2: {N_COPIES} rotating weight copies "
+                  f"({N_COPIES * weight_bytes / 1e6:.0f} MB) in a CUDA graph",
+            "parallelism": f"replicas x{ws} (independent problems, no collective)",
+        },
+        "roofline": {
+            "bound": "hbm", "achieved": round(dec_achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(dec_achieved / hbm_peak, 4),
+            "traffic": measured_traffic("decode_kernel", ["decode.cuh", "common.cuh"]),
+            "kernel": "w8::decode::decode_kernel<1>",
+            "algorithmic_bytes_per_launch": alg_bytes,
+            "peak_source": f"{peak_src} hbm_gbs",
+        },
+        "prefill": {
+            "metric": "TFLOP/s (M=2048, 4096x27392)", "value": round(pf_tflops, 1), "unit": "TFLOP/s",
+            "us_per_call": round(pf_s * 1e6, 2),
+            "roofline": {"bound": "tensor", "achieved": round(pf_tflops, 1), "peak": tf_peak,
+                         "unit": "TFLOP/s", "frac": round(pf_tflops / tf_peak, 4),
+                         "traffic": measured_traffic("prefill_kernel", ["prefill.cuh", "common.cuh"]),
+                         "peak_source": f"{peak_src} bf16_tflops (burst) x fp16/bf16 nominal ratio 1"},
+        },
+        "quantize": {
+            "us_per_call": round(t_q * 1e6, 2), "algorithmic_GBps": round(q_bytes / t_q / 1e9, 1),
+            "frac_hbm": round(q_bytes / t_q / 1e9 / hbm_peak, 4), "bit_identical_rerun": same,
+            "traffic": measured_traffic("quantize_kernel", ["quantize.cuh", "common.cuh"]),
+        },
+        "prepack": {"us_per_call": round(t_pk * 1e6, 2),
+                    "algorithmic_GBps": round(pk_bytes / t_pk / 1e9, 1)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
+                "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()),
+                "how": "public API call per step with pinned-host X->device and Y->host copies, "
+                       "graph-replayed"},
+        "gpu_launches": steps_done,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    for g in (g_dec, g_pf, g_q, g_pk, g_e2e):
+        del g
+    return out
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_slab(cols: int, seed: int):
+    import synthetic
+    tid = synthetic.tensor_id(2, 0, 0, 0)
+    W = synthetic.weights(K_DIM, N_DIM, seed, tid, outlier_frac=0.001)
+    X = synthetic.activations(M_DECODE, K_DIM, seed, tid + 1)
+    return X, np.ascontiguousarray(W[:, :cols])
+
+
+def cpu_baseline(seconds: float):
+    """The CPU oracle as it stands (plain C, one thread) on a column slab of
+    the decode workload, repeated for about `seconds`."""
+    import oracle
+    cols = 4096
+    X, Ws = oracle_slab(cols, 20231002)
+    q, s = oracle.quantize(Ws)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.linear(X, q, s)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    gbps = K_DIM * cols * reps / el / 1e9
+    return {"value": round(gbps, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} x oracle_linear M=1 on a 4096x{cols} column slab of the "
+                      f"4096x27392 weight ({el:.1f} s, host has {os.cpu_count()} cores)"}
+
+
+def run_reference(args):
+    import oracle
+    cols = args.ref_cols
+    X, Ws = oracle_slab(cols, 20231002)
+    q, s = oracle.quantize(Ws)
+    for _ in range(args.warmup):
+        oracle.linear(X, q, s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.linear(X, q, s)
+    el = time.perf_counter() - t0
+    value = K_DIM * cols * args.steps / el / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_DECODE, "K": K_DIM, "N": N_DIM,
+                   "sample": f"each step: oracle linear over a 4096x{cols} column slab"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} steps x 4096x{cols} weight slab, M=1"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30000)
+    ap.add_argument("--warmup", type=int, default=60)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--prefill-reps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-cols", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    ws, rank, local = dist_setup()
+    out = run_native(args, ws, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -77,7 +77,8 @@ typedef enum { W8_F32 = 0, W8_F16 = 1 } w8_dtype;
  *           W8_F16); fp16 is widened exactly to fp32 first.
  *   q       [K, N] int8 output codes in [-127, 127].
  *   scales  [N] fp16 output scales.
- *   K >= 1; N >= 0 with N % 8 == 0 (N == 0 is a no-op).
+ *   K >= 1; N >= 0 with N % 8 == 0 (N == 0 is a no-op and the pointers
+ *   may then be NULL).
  * The result is bit-exact: fp32 divisions are IEEE round-to-nearest, the
  * fp32 -> fp16 and fp32 -> int conversions round half to even, fp16
  * subnormal scales are kept.  Inputs must be finite.
@@ -135,12 +136,15 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *   scales     [N] fp16 per-channel scales (w8_quantize_per_channel output).
  *   bias       [N] fp16 or NULL.
  *   Y          [M, N] fp16 output; must not overlap X, packed or scales.
- *   M >= 0 (0 is a no-op); K >= 1 with K % 8 == 0; N >= 1 with N % 8 == 0.
+ *   M >= 0 (0 is a no-op; X and Y may then be NULL); K >= 1 with
+ *   K % 8 == 0; N >= 1 with N % 8 == 0.
  *   workspace  device scratch of at least w8a16_workspace_bytes(M, K, N)
  *              bytes (may be NULL when that is 0).  It must be all zero
- *              before its first use; every call leaves it ready for the
- *              next one.  Calls sharing one workspace must not run
- *              concurrently on the device.
+ *              before its first use; every call that completes leaves it
+ *              ready for the next one, whatever the next call's shape.
+ *              Calls sharing one workspace must not run concurrently on
+ *              the device.  After a call whose device wait ran out (see
+ *              w8_device_status) the workspace must be zeroed again.
  * Kernel choice (internal): M <= 16 streams the weight once with a
  * split-K decode kernel (HBM-bound); larger M runs a tcgen05 tensor-core
  * kernel with the widened weight tile held in tensor memory.

@@ -45,7 +45,7 @@ struct Cfg {
     static constexpr int kPartialFloats = kConsumerWarps * 4 * MT * 32;   // per slot
 };
 
-// Workspace: [counters: NB int32, padded to 256 B][partials: 2G slots]
+// Workspace: [partials: 2 slots per SM][counters: one int32 per channel block]
 constexpr int kMaxPartialFloats = Cfg<2>::kPartialFloats;
 
 struct Params {

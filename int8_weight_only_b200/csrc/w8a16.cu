@@ -181,17 +181,17 @@ const char *w8_error_string(int status) {
 
 int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
                             uint16_t *scales, void *stream) {
-    if (!W || !q || !scales) return W8_ERR_NULL;
     if (w_dtype != W8_F32 && w_dtype != W8_F16) return W8_ERR_DTYPE;
     if (K < 1 || N < 0 || N % 8 != 0 || K > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX * 8)
         return W8_ERR_SHAPE;
+    if (N == 0) return W8_OK;   // nothing to read or write: pointers may be NULL
+    if (!W || !q || !scales) return W8_ERR_NULL;
     if (!aligned16(W) || !aligned16(q) || !aligned16(scales)) return W8_ERR_ALIGN;
     const size_t welem = w_dtype == W8_F32 ? 4 : 2;
     if (overlap(W, (size_t)K * N * welem, q, (size_t)K * N) ||
         overlap(W, (size_t)K * N * welem, scales, (size_t)N * 2) ||
         overlap(q, (size_t)K * N, scales, (size_t)N * 2))
         return W8_ERR_ALIAS;
-    if (N == 0) return W8_OK;
     DeviceInfo *d = nullptr;
     int rc = device_info(&d);
     if (rc != W8_OK) return rc;
@@ -212,12 +212,14 @@ size_t w8_prepacked_bytes(int64_t K, int64_t N) {
     return (size_t)cdiv(N, W8_TILE_N) * (size_t)cdiv(K, W8_TILE_K) * W8_TILE_BYTES;
 }
 
-static int pack_args(const void *a, const void *b, int64_t K, int64_t N) {
-    if (!a || !b) return W8_ERR_NULL;
+// q is the [K, N] code matrix (K*N bytes), packed the tiled copy
+// (w8_prepacked_bytes(K, N) bytes, larger than K*N for ragged shapes).
+static int pack_args(const void *q, const void *packed, int64_t K, int64_t N) {
+    if (!q || !packed) return W8_ERR_NULL;
     if (K < 1 || N < 1 || N % 8 != 0 || cdiv(K, 64) > 65535 * 1024LL || cdiv(N, 128) > 65535)
         return W8_ERR_SHAPE;
-    if (!aligned16(a) || !aligned16(b)) return W8_ERR_ALIGN;
-    if (overlap(a, w8_prepacked_bytes(K, N), b, w8_prepacked_bytes(K, N))) return W8_ERR_ALIAS;
+    if (!aligned16(q) || !aligned16(packed)) return W8_ERR_ALIGN;
+    if (overlap(q, (size_t)K * (size_t)N, packed, w8_prepacked_bytes(K, N))) return W8_ERR_ALIAS;
     return W8_OK;
 }
 
@@ -234,7 +236,7 @@ int w8_prepack(const int8_t *q, int64_t K, int64_t N, uint8_t *packed, void *str
 }
 
 int w8_unpack(const uint8_t *packed, int64_t K, int64_t N, int8_t *q, void *stream) {
-    int rc = pack_args(packed, q, K, N);
+    int rc = pack_args(q, packed, K, N);
     if (rc != W8_OK) return rc;
     DeviceInfo *d = nullptr;
     if ((rc = device_info(&d)) != W8_OK) return rc;
@@ -248,12 +250,18 @@ int w8_unpack(const uint8_t *packed, int64_t K, int64_t N, int8_t *q, void *stre
 // Decode split: one CTA per SM (never more CTAs than tiles).
 static int decode_grid(int sms, int64_t T) { return (int)std::max<int64_t>(1, std::min<int64_t>(T, sms)); }
 
+// Decode workspace: [partials: 2 slots per SM][counters: one int32 per 128
+// channels].  The partial area has the same size for every shape on a
+// device, so the counters always start at the same offset: a workspace that
+// served one shape (and was left with zero counters) serves any other.
+static size_t decode_partials_bytes(int sms) {
+    return (size_t)2 * sms * decode::kMaxPartialFloats * sizeof(float);
+}
+
 static size_t decode_workspace(int sms, int64_t K, int64_t N) {
-    const int64_t NB = cdiv(N, 128), T = NB * cdiv(K, 64);
-    const int G = decode_grid(sms, T);
-    const size_t counters = (size_t)cdiv(NB * 4, 256) * 256;
-    const size_t partials = (size_t)2 * G * decode::kMaxPartialFloats * sizeof(float);
-    return counters + partials;
+    (void)K;
+    const int64_t NB = cdiv(N, 128);
+    return decode_partials_bytes(sms) + (size_t)cdiv(NB * 4, 256) * 256;
 }
 
 size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N) {
@@ -266,10 +274,12 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N) {
 int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
                  const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
                  void *workspace, size_t workspace_bytes, void *stream) {
-    if (!X || !packed || !scales || !Y) return W8_ERR_NULL;
     if (M < 0 || K < 1 || N < 1 || K % 8 != 0 || N % 8 != 0 || M > (int64_t)INT32_MAX ||
         K > (int64_t)INT32_MAX || cdiv(K, 64) > INT32_MAX)
         return W8_ERR_SHAPE;
+    if (!packed || !scales) return W8_ERR_NULL;
+    if (M == 0) return W8_OK;   // empty batch: X and Y may be NULL
+    if (!X || !Y) return W8_ERR_NULL;
     if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(Y) ||
         (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
         return W8_ERR_ALIGN;
@@ -278,7 +288,6 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
         overlap(Y, ybytes, packed, w8_prepacked_bytes(K, N)) ||
         overlap(Y, ybytes, scales, (size_t)N * 2) || (bias && overlap(Y, ybytes, bias, (size_t)N * 2)))
         return W8_ERR_ALIAS;
-    if (M == 0) return W8_OK;
     DeviceInfo *d = nullptr;
     int rc = device_info(&d);
     if (rc != W8_OK) return rc;
@@ -301,9 +310,9 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
         p.scales = scales;
         p.bias = bias;
         p.Y = Y;
-        p.counters = static_cast<int *>(workspace);
-        p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                               (size_t)cdiv(NB * 4, 256) * 256);
+        p.partials = static_cast<float *>(workspace);
+        p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) +
+                                             decode_partials_bytes(d->sms));
         p.M = (int)M;
         p.N = N;
         p.KB = KB;

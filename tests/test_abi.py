@@ -70,6 +70,7 @@ def test_quantize_rejects_bad_arguments(w8lib):
     assert q(ctypes.c_void_p(0x10004), 0, 4, 8, B, C, None) == -3
     assert q(A, 0, 4, 8, ctypes.c_void_p(0x10000 + 16), C, None) == -8   # q inside W
     assert q(A, 0, 4, 0, B, C, None) == 0                                   # empty: no-op
+    assert q(None, 0, 4, 0, None, None, None) == 0                          # empty tensors
 
 
 def test_pack_rejects_bad_arguments(w8lib):
@@ -79,6 +80,16 @@ def test_pack_rejects_bad_arguments(w8lib):
         assert fn(A, 64, 100, B, None) == -2
         assert fn(A, 64, 128, ctypes.c_void_p(0x20000008), None) == -3
         assert fn(A, 64, 128, ctypes.c_void_p(0x10000 + 4096), None) == -8
+    # ragged shape: q holds K*N = 8840 bytes, the packed copy 4 tiles; a
+    # packed buffer that starts right after q does not overlap it
+    K, N = 65, 136
+    qa, pk = 0x10000, 0x10000 + ((K * N + 15) // 16) * 16
+    assert w8lib.w8_prepacked_bytes(K, N) > K * N
+    # valid arguments reach the CUDA runtime (-6 without a device) instead
+    # of being refused as overlapping
+    assert w8lib.w8_prepack(ctypes.c_void_p(qa), K, N, ctypes.c_void_p(pk), None) != -8
+    assert w8lib.w8_unpack(ctypes.c_void_p(pk), K, N, ctypes.c_void_p(qa), None) != -8
+    assert w8lib.w8_prepack(ctypes.c_void_p(qa), K, N, ctypes.c_void_p(pk - 16), None) == -8
 
 
 def test_linear_rejects_bad_arguments(w8lib):
@@ -92,6 +103,8 @@ def test_linear_rejects_bad_arguments(w8lib):
     assert L(A, B, C, ctypes.c_void_p(0x3), D, 1, 64, 128, E, 1 << 20, None) == -3
     assert L(A, B, C, None, ctypes.c_void_p(0x10000 + 64), 1, 64, 128, E, 1 << 20, None) == -8
     assert L(A, B, C, None, D, 0, 64, 128, E, 1 << 20, None) == 0        # M == 0: no-op
+    assert L(None, B, C, None, None, 0, 64, 128, None, 0, None) == 0     # empty X, Y
+    assert L(None, None, C, None, None, 0, 64, 128, None, 0, None) == -1
 
 
 def test_valid_call_without_gpu_fails_loudly(w8lib):
