@@ -58,7 +58,9 @@ typedef enum {
     W8_ERR_CUDA = -6,       /* a CUDA runtime call or launch failed */
     W8_ERR_TIMEOUT = -7,    /* a bounded device wait ran out (see w8_device_status) */
     W8_ERR_ALIAS = -8,      /* the output overlaps an input */
-    W8_ERR_DEVICE = -9      /* the current device is not sm_100 */
+    W8_ERR_DEVICE = -9,     /* the current device is not sm_100 */
+    W8_ERR_LIMIT = -10      /* a size exceeds the fixed scratch of
+                               w8a16_linear_decode_static */
 } w8_status;
 
 typedef enum { W8_F32 = 0, W8_F16 = 1 } w8_dtype;
@@ -155,6 +157,41 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
 int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
                  const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * w8a16_linear_decode_static -- the decode path of w8a16_linear (M <= 16)
+ * without a caller-provided workspace.  The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory, such
+ * as an operator plugged into a host framework whose fixed signature has no
+ * workspace argument, or a serving loop whose device memory is planned up
+ * front by another allocator and where a cudaMalloc would synchronize the
+ * device.  Their inputs and outputs are still passed in.
+ *
+ * The split-K scratch (fp32 partial sums and per-block counters) lives in
+ * one array of W8_STATIC_SCRATCH_BYTES bytes of static device memory inside
+ * this library; every GPU that loads the library holds it until the
+ * process exits.  Nothing is allocated or freed by the call.
+ *
+ *   Arguments and results as for w8a16_linear, with these limits:
+ *   1 <= M <= 16 (M == 0 is a no-op), N <= W8_STATIC_MAX_N, and the device
+ *   has at most W8_STATIC_MAX_SMS multiprocessors.  Beyond them the call
+ *   returns W8_ERR_LIMIT before anything is launched.
+ *   Each call first clears the counters it uses (cudaMemsetAsync on
+ *   `stream`), so leftovers of an earlier call, finished or not, do no harm.
+ *   All calls share the one array: calls that can overlap on the GPU (on
+ *   different streams, or from different host threads) race and must be
+ *   ordered by the caller.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   outside any stream capture.
+ * Errors: those of w8a16_linear except W8_ERR_WORKSPACE, plus W8_ERR_LIMIT.
+ */
+#define W8_STATIC_MAX_SMS 160
+#define W8_STATIC_MAX_N (1 << 20)
+#define W8_STATIC_SCRATCH_BYTES (2 * W8_STATIC_MAX_SMS * 8192 + (W8_STATIC_MAX_N / 128) * 4)
+int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
+                               const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
+                               void *stream);
 
 /* w8_error_string -- static text for a w8_status value. */
 const char *w8_error_string(int status);

@@ -19,7 +19,7 @@ import threading
 
 __all__ = [
     "W8Error", "load_library", "library_path", "quantize", "prepack", "unpack",
-    "prepacked_bytes", "workspace_bytes", "linear", "W8A16Linear", "device_status",
+    "prepacked_bytes", "workspace_bytes", "linear", "linear_decode_static", "W8A16Linear", "device_status",
     "test_bounded_wait", "STATUS",
 ]
 
@@ -29,7 +29,7 @@ _LIB_PATH = os.path.join(_HERE, "libw8a16.so")
 STATUS = {
     0: "W8_OK", -1: "W8_ERR_NULL", -2: "W8_ERR_SHAPE", -3: "W8_ERR_ALIGN", -4: "W8_ERR_DTYPE",
     -5: "W8_ERR_WORKSPACE", -6: "W8_ERR_CUDA", -7: "W8_ERR_TIMEOUT", -8: "W8_ERR_ALIAS",
-    -9: "W8_ERR_DEVICE",
+    -9: "W8_ERR_DEVICE", -10: "W8_ERR_LIMIT",
 }
 W8_F32, W8_F16 = 0, 1
 
@@ -68,12 +68,14 @@ def load_library():
         lib.w8a16_workspace_bytes.argtypes = [i64, i64, i64]
         lib.w8a16_workspace_bytes.restype = sz
         lib.w8a16_linear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp]
+        lib.w8a16_linear_decode_static.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
         lib.w8_error_string.argtypes = [i32]
         lib.w8_error_string.restype = ctypes.c_char_p
         lib.w8_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         lib.w8_test_bounded_wait.argtypes = [ctypes.c_uint64, vp]
         lib.w8_version.argtypes = []
         for f in ("w8_quantize_per_channel", "w8_prepack", "w8_unpack", "w8a16_linear",
+                  "w8a16_linear_decode_static",
                   "w8_device_status", "w8_test_bounded_wait", "w8_version"):
             getattr(lib, f).restype = i32
         _lib = lib
@@ -202,6 +204,29 @@ def linear(X, packed, scales, bias=None, out=None, workspace=None):
         ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
         _check(lib.w8a16_linear(_ptr(X), _ptr(packed), _ptr(scales), _ptr(bias), _ptr(out),
                                 M, K, N, _ptr(ws), ws_bytes, _stream(X.device)), "w8a16_linear")
+    return out
+
+
+def linear_decode_static(X, packed, scales, bias=None, out=None):
+    """Decode-path linear (M <= 16) that needs no workspace: its scratch is a
+    fixed array of static device memory inside the library.  For callers
+    that cannot allocate device memory (an operator inside a host framework
+    whose signature has no workspace argument, or a loop whose memory is
+    planned up front by another allocator).  Calls that may overlap on the
+    GPU share that array and must be ordered by the caller."""
+    torch = _torch()
+    lib = load_library()
+    _need_cuda(X, "X")
+    if X.dim() != 2 or X.dtype != torch.float16:
+        raise ValueError("X must be [M, K] float16")
+    M, K = X.shape
+    N = scales.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    with torch.cuda.device(X.device):
+        _check(lib.w8a16_linear_decode_static(_ptr(X), _ptr(packed), _ptr(scales), _ptr(bias),
+                                              _ptr(out), M, K, N, _stream(X.device)),
+               "w8a16_linear_decode_static")
     return out
 
 

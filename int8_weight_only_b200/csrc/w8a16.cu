@@ -175,6 +175,9 @@ const char *w8_error_string(int status) {
         case W8_ERR_TIMEOUT: return "a bounded device wait ran out";
         case W8_ERR_ALIAS: return "output overlaps an input";
         case W8_ERR_DEVICE: return "current device is not sm_100 (B200)";
+        case W8_ERR_LIMIT:
+            return "size beyond the fixed scratch of w8a16_linear_decode_static "
+                   "(needs 1 <= M <= 16, N <= 2^20, at most 160 SMs)";
         default: return "unknown status";
     }
 }
@@ -378,3 +381,102 @@ int w8_device_status(void *stream, uint32_t *out) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free decode
+// w8a16_linear_decode_static: the decode kernel with its split-K scratch in
+// a fixed array of static device memory instead of a caller workspace, for
+// callers that cannot allocate device memory.  Layout of the array:
+// [fp32 partials: 2 slots x up to W8_STATIC_MAX_SMS CTAs][int32 counters:
+// one per 128-channel block, up to W8_STATIC_MAX_N / 128].
+namespace {
+constexpr size_t kStaticPartialBytes =
+    (size_t)2 * W8_STATIC_MAX_SMS * decode::kMaxPartialFloats * sizeof(float);
+constexpr size_t kStaticCounterBytes = (size_t)(W8_STATIC_MAX_N / 128) * sizeof(int);
+static_assert(kStaticPartialBytes + kStaticCounterBytes == (size_t)W8_STATIC_SCRATCH_BYTES,
+              "header size of the static scratch");
+}  // namespace
+
+// One copy per device that loads this library, zero at load, kept until exit.
+static __device__ __align__(256) uint8_t g_decode_scratch[W8_STATIC_SCRATCH_BYTES];
+
+namespace {
+// Device address of g_decode_scratch, looked up once per device.  In host
+// code the array's name is only a host-side stand-in, never a device
+// address, so kernels get this pointer instead.
+void *g_scratch_ptr[kMaxDevices];
+std::mutex g_scratch_mu;
+
+int static_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W8_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return W8_ERR_CUDA;
+        }
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return W8_OK;
+}
+}  // namespace
+
+extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *packed,
+                                          const uint16_t *scales, const uint16_t *bias, uint16_t *Y,
+                                          int64_t M, int64_t K, int64_t N, void *stream) {
+    if (M < 0 || K < 1 || N < 1 || K % 8 != 0 || N % 8 != 0 || K > (int64_t)INT32_MAX ||
+        cdiv(K, 64) > INT32_MAX)
+        return W8_ERR_SHAPE;
+    if (M > 16 || N > (int64_t)W8_STATIC_MAX_N) return W8_ERR_LIMIT;
+    if (!packed || !scales) return W8_ERR_NULL;
+    if (M == 0) return W8_OK;
+    if (!X || !Y) return W8_ERR_NULL;
+    if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(Y) ||
+        (bias && !aligned16(bias)))
+        return W8_ERR_ALIGN;
+    const size_t ybytes = (size_t)M * N * 2;
+    if (overlap(Y, ybytes, X, (size_t)M * K * 2) ||
+        overlap(Y, ybytes, packed, w8_prepacked_bytes(K, N)) ||
+        overlap(Y, ybytes, scales, (size_t)N * 2) || (bias && overlap(Y, ybytes, bias, (size_t)N * 2)))
+        return W8_ERR_ALIAS;
+    DeviceInfo *d = nullptr;
+    int rc = device_info(&d);
+    if (rc != W8_OK) return rc;
+    if (d->sms > W8_STATIC_MAX_SMS) return W8_ERR_LIMIT;
+    void *scratch = nullptr;
+    if ((rc = static_scratch(&scratch)) != W8_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int KB = (int)cdiv(K, 64);
+    const int64_t NB = cdiv(N, 128);
+    int *counters = reinterpret_cast<int *>(static_cast<uint8_t *>(scratch) + kStaticPartialBytes);
+    // the counters must start at zero; an earlier call that gave up a wait
+    // may have left some set
+    if (cudaMemsetAsync(counters, 0, (size_t)NB * sizeof(int), st) != cudaSuccess) {
+        cudaGetLastError();
+        return W8_ERR_CUDA;
+    }
+    const int MT = M <= 8 ? 1 : 2;
+    CUtensorMap map;
+    rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64, 8 * MT,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != W8_OK) return rc;
+    decode::Params p;
+    p.packed = packed;
+    p.scales = scales;
+    p.bias = bias;
+    p.Y = Y;
+    p.partials = static_cast<float *>(scratch);
+    p.counters = counters;
+    p.M = (int)M;
+    p.N = N;
+    p.KB = KB;
+    p.T = NB * KB;
+    p.G = decode_grid(d->sms, p.T);
+    if (MT == 1)
+        decode::decode_kernel<1><<<p.G, decode::kThreads, decode::Cfg<1>::kSmemBytes, st>>>(map, p);
+    else
+        decode::decode_kernel<2><<<p.G, decode::kThreads, decode::Cfg<2>::kSmemBytes, st>>>(map, p);
+    return launch_status();
+}
