@@ -338,10 +338,14 @@ def run_native(args, ws, rank, local):
         "prefill": {
             "metric": "TFLOP/s (M=2048, 4096x27392)", "value": round(pf_tflops, 1), "unit": "TFLOP/s",
             "us_per_call": round(pf_s * 1e6, 2),
-            "roofline": {"bound": "tensor", "achieved": round(pf_tflops, 1), "peak": tf_peak,
-                         "unit": "TFLOP/s", "frac": round(pf_tflops / tf_peak, 4),
+            # the prefill timed region is a long back-to-back loop under the
+            # power cap, the condition of the sustained GEMM measurement
+            "roofline": {"bound": "tensor", "achieved": round(pf_tflops, 1), "peak": tf_sustained,
+                         "unit": "TFLOP/s", "frac": round(pf_tflops / tf_sustained, 4),
+                         "frac_of_burst": round(pf_tflops / tf_peak, 4),
                          "traffic": measured_traffic("prefill_kernel", ["prefill.cuh", "common.cuh"]),
-                         "peak_source": f"{peak_src} bf16_tflops (burst) x fp16/bf16 nominal ratio 1"},
+                         "peak_source": f"{peak_src} bf16_tflops_sustained (cuBLAS loop under the power cap) "
+                                        f"x fp16/bf16 nominal ratio 1; burst {tf_peak}"},
         },
         "quantize": {
             "us_per_call": round(t_q * 1e6, 2), "algorithmic_GBps": round(q_bytes / t_q / 1e9, 1),
@@ -363,6 +367,40 @@ def run_native(args, ws, rank, local):
     for g in (g_dec, g_pf, g_q, g_pk, g_e2e):
         del g
     return out
+
+
+# ------------------------------------------------------------------ profiling driver
+def run_profile(args):
+    """A few plain launches of one kernel on the bench's workload, for ncu
+    captures (no graphs, no timing).  Two packed-weight copies alternate so
+    the weight (2 x 112 MB) is not served from L2."""
+    import torch
+    import synthetic
+    import int8_weight_only_b200 as w8
+    from int8_weight_only_b200 import build as w8build
+
+    w8build.build()
+    w8.load_library()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    tid = synthetic.tensor_id(2, 0, 0, 0)
+    W = torch.from_numpy(synthetic.weights(K_DIM, N_DIM, synthetic.SEED, tid, outlier_frac=0.001)).to(device)
+    q, scales = w8.quantize(W)
+    copies = [w8.prepack(q) for _ in range(2)]
+    M = {"decode": M_DECODE, "decode16": 16, "prefill": M_PREFILL}.get(args.profile, M_DECODE)
+    X = torch.from_numpy(synthetic.activations(M, K_DIM, synthetic.SEED, tid + 1)).to(device)
+    Y = torch.empty((M, N_DIM), dtype=torch.float16, device=device)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        if args.profile in ("decode", "decode16", "prefill"):
+            w8.linear(X, copies[i % 2], scales, out=Y)
+        elif args.profile == "quantize":
+            w8.quantize(W, q=q, scales=scales)
+        elif args.profile == "prepack":
+            w8.prepack(q, out=copies[i % 2])
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "launches": args.steps, "M": M, "K": K_DIM, "N": N_DIM}))
+    return 0
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -431,7 +469,11 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-cols", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["decode", "decode16", "prefill", "quantize", "prepack"],
+                    help="run --steps plain launches of one kernel (for ncu) and exit")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile(args)
     if args.warmup < 3:
         args.warmup = 3
 

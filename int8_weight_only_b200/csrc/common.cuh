@@ -22,6 +22,8 @@ enum WaitSite : unsigned {
     SITE_Q_LOAD = 0x10,
     SITE_DEC_EMPTY = 0x20,
     SITE_DEC_FULL = 0x21,
+    SITE_DEC_FIX = 0x22,
+    SITE_DEC_DRAIN = 0x23,
     SITE_PF_EMPTY = 0x30,
     SITE_PF_FULL_CVT = 0x31,
     SITE_PF_FULL_MMA = 0x32,
@@ -30,6 +32,7 @@ enum WaitSite : unsigned {
     SITE_PF_DEMPTY = 0x35,
     SITE_PF_DFULL = 0x36,
     SITE_PF_DRAIN = 0x37,
+    SITE_PF_XEMPTY = 0x38,
     SITE_SELFTEST = 0xEE,
 };
 
@@ -44,6 +47,32 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// Let the next kernel in the stream (launched with programmatic stream
+// serialization) start its prologue while this grid is still running.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the previous grid in the stream has completed and its memory
+// operations are visible (returns at once when there is none).
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Bring [src, src + bytes) into L2 without touching shared memory (16-byte
+// aligned address, size a multiple of 16).  Safe before pdl_wait: L2 is
+// coherent, so a later write by the previous grid simply updates the lines.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// ---------------------------------------------------------------- global memory ordering
+// Load with acquire semantics at GPU scope.
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 // ---------------------------------------------------------------- smem
@@ -96,15 +125,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned site,
                                           unsigned long long limit_ns = kWaitLimitNs) {
     const uint32_t a = smem_u32(bar);
+    // the clock is read only once a wait is long (it costs time in the
+    // streaming loops, where almost every wait ends within these tries)
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < 512; ++i) {
         if (mbar_try_wait(a, parity)) return true;
     }
     const unsigned long long t0 = globaltimer_ns();
 #pragma unroll 1
     while (true) {
 #pragma unroll 1
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 512; ++i) {
             if (mbar_try_wait(a, parity)) return true;
         }
         if (globaltimer_ns() - t0 > limit_ns) {

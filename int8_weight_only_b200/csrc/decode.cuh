@@ -16,11 +16,19 @@
 //    pattern of 1024, then one fp16x2 subtraction) and accumulate in fp32
 //    with mma.sync m16n8k16 (channels as the MMA rows, tokens as its 8 or
 //    16 columns), so conversion plus multiply-add stay a small fraction of
-//    the issue budget even at 16 tokens.
-//  - A channel block whose K range is split between CTAs is finished by the
-//    last CTA to arrive (an atomic counter per block, reset by that CTA):
-//    it adds the fp32 partials of all contributors in CTA order, so the
-//    result does not depend on arrival order, then applies scale and bias.
+//    the issue budget even at 16 tokens.  The stage's tiles are unrolled and
+//    each 16-wide k slice has its own accumulator, so the mma results do not
+//    form one long dependency chain.
+//  - Only a CTA's first and last channel block can be split with other
+//    CTAs.  A split part is published to the workspace (fp32 partial sums,
+//    one fence, an atomic counter per block) as soon as it is done, and the
+//    last contributor to arrive adds all parts in CTA order (so the result
+//    does not depend on arrival order), applies scale and bias and resets
+//    the counter.  The common two-way split (this CTA streams the first K
+//    blocks of its last channel block last, the next CTA streams the rest
+//    first) short-cuts this: when this CTA reaches that block the next CTA
+//    has normally published already, so its part is loaded into registers
+//    during the stream and the block is finished with no fence or atomic.
 #pragma once
 
 #include "common.cuh"
@@ -57,17 +65,19 @@ struct Params {
     float *partials;
     int M;
     int64_t N;
-    int KB;      // ceil(K / 64)
-    int64_t T;   // tiles
-    int G;       // CTAs
+    int KB;        // ceil(K / 64)
+    uint32_t T;    // tiles; the host guarantees T * (G + 1) < 2^32
+    uint32_t G;    // CTAs
 };
 
-__device__ __forceinline__ int64_t range_start(int i, int64_t T, int G) {
-    return (int64_t)i * T / G;
+// Stream-K split in 32-bit arithmetic (64-bit division is a long software
+// sequence and sat on the critical path of every stage).
+__device__ __forceinline__ uint32_t range_start(uint32_t i, uint32_t T, uint32_t G) {
+    return i * T / G;
 }
 // CTA whose range holds tile t.
-__device__ __forceinline__ int owner_of(int64_t t, int64_t T, int G) {
-    return (int)(((t + 1) * (int64_t)G - 1) / T);
+__device__ __forceinline__ uint32_t owner_of(uint32_t t, uint32_t T, uint32_t G) {
+    return ((t + 1) * G - 1) / T;
 }
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -87,12 +97,12 @@ __device__ __forceinline__ uint16_t out_f16(float acc, float s, float b) {
 // mt, acc[mt] = Y^T[n][m] at n = 16w+g (+8 for elements 2,3) and
 // m = 8mt + 2t (+1 for elements 1,3).
 template <int MT>
-__device__ __forceinline__ void store_y(const Params &p, int64_t b, int warp, int lane,
+__device__ __forceinline__ void store_y(const Params &p, uint32_t b, int warp, int lane,
                                         const float (&acc)[MT][4]) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-        const int64_t n = b * 128 + 16 * warp + g + 8 * half;
+        const int64_t n = (int64_t)b * 128 + 16 * warp + g + 8 * half;
         if (n >= p.N) continue;
         const float s = __half2float(__ushort_as_half(p.scales[n]));
         const float bb = p.bias ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
@@ -107,6 +117,16 @@ __device__ __forceinline__ void store_y(const Params &p, int64_t b, int warp, in
     }
 }
 
+// Sum the four per-k-slice accumulators of each token tile.
+template <int MT>
+__device__ __forceinline__ void fold(const float (&acc)[MT][4][4], float (&out)[MT][4]) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            out[mt][e] = (acc[mt][0][e] + acc[mt][1][e]) + (acc[mt][2][e] + acc[mt][3][e]);
+}
+
 template <int MT>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
@@ -116,13 +136,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ uint64_t full[kStages], empty[kStages];
     __shared__ uint64_t fix_bar;
-    __shared__ int last_flag;
+    __shared__ int last_flag[2];   // [0]: partner part ready; [1]: last contributor
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int cta = blockIdx.x;
-    const int64_t t_begin = range_start(cta, p.T, p.G);
-    const int64_t t_end = range_start(cta + 1, p.T, p.G);
+    const uint32_t cta = blockIdx.x;
+    const uint32_t KB = (uint32_t)p.KB;
+    const uint32_t t_begin = range_start(cta, p.T, p.G);
+    const uint32_t t_end = range_start(cta + 1, p.T, p.G);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -134,31 +155,51 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         prefetch_tensormap(&tmap_x);
     }
     __syncthreads();
+    // The next call may start as soon as SMs free up; it only touches this
+    // call's data after its own pdl_wait.
+    pdl_launch_dependents();
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
+            // The weights are not written by the previous kernel in any
+            // sane use, but only an L2 prefetch (never stale) runs before
+            // the wait: the first ring's worth of this CTA's range.
+            const uint32_t pre_tiles = min(t_end - t_begin, (uint32_t)(kStages * kTilesPerStage));
+            prefetch_l2(p.packed + (size_t)t_begin * kTileBytes, pre_tiles * kTileBytes);
+            pdl_wait();
             const uint64_t policy = policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
-            for (int64_t t = t_begin; t < t_end;) {
-                const int kb = (int)(t % p.KB);
-                const int cnt = (int)min64(kTilesPerStage, min64(t_end - t, p.KB - kb));
+            int issued = 0;
+            uint32_t kb = t_begin % KB;
+            for (uint32_t t = t_begin; t < t_end;) {
+                const int cnt = (int)min(min((uint32_t)kTilesPerStage, t_end - t), KB - kb);
                 if (!mbar_wait(&empty[stage], phase ^ 1u, SITE_DEC_EMPTY)) break;
                 uint8_t *ws = base + stage * C::kStageBytes;
                 uint8_t *xs = ws + kStageW;
                 mbar_arrive_expect_tx(&full[stage], cnt * (kTileBytes + C::kXBoxBytes));
-                bulk_g2s_hint(ws, p.packed + t * kTileBytes, cnt * kTileBytes, &full[stage], policy);
+                bulk_g2s_hint(ws, p.packed + (size_t)t * kTileBytes, cnt * kTileBytes, &full[stage], policy);
                 for (int j = 0; j < cnt; ++j)
-                    tma_load_2d(xs + j * C::kXBoxBytes, &tmap_x, (kb + j) * 64, 0, &full[stage]);
+                    tma_load_2d(xs + j * C::kXBoxBytes, &tmap_x, (int)(kb + j) * 64, 0, &full[stage]);
                 t += cnt;
+                kb += cnt;
+                if (kb == KB) kb = 0;
+                ++issued;
                 if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            }
+            // every copy this CTA issued has landed before the CTA can exit
+            // (normally long since consumed; matters only after a timeout)
+            for (int i = 0; i < kStages && i < issued; ++i) {
+                if (--stage < 0) { stage = kStages - 1; phase ^= 1u; }
+                mbar_wait(&full[stage], phase, SITE_DEC_DRAIN, 10000000ull);
             }
         }
         return;
     }
 
     // ---------------------------------------------------------- consumers
+    pdl_wait();   // before any global access of this grid's consumers
     const int g = lane >> 2, tq = lane & 3;
     const int h = (g >> 1) & 3;                     // chunk swizzle of rows 16w+g, 16w+g+8
     const int row_lo = 16 * warp + g;
@@ -172,109 +213,172 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         x_off[mt][1] = m * 128 + (((2 * tq + 1) ^ (m & 7)) << 4);
     }
 
-    float acc[MT][4];
+    // one accumulator per 16-wide k slice of the tile: four independent
+    // mma chains instead of one
+    float acc[MT][4][4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][e] = 0.0f;
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][jj][e] = 0.0f;
+
+    uint32_t fix_phase = 0;
+    // all 256 consumer threads meet (bounded); false if the wait ran out
+    auto consumers_sync = [&]() -> bool {
+        mbar_arrive(&fix_bar);
+        const bool ok = mbar_wait(&fix_bar, fix_phase, SITE_DEC_FIX);
+        fix_phase ^= 1u;
+        return ok;
+    };
+
+    // The last channel block of this CTA, when only its first K blocks are
+    // here and the rest belongs to the next CTA alone (a two-way split with
+    // this CTA holding the part that is streamed last): the next CTA
+    // publishes its part early in its stream, so this CTA can usually pick
+    // it up while streaming its own part and finish the block without any
+    // fence or atomic at the end.
+    const uint32_t first_b = t_begin / KB;
+    const uint32_t last_b = (t_end - 1) / KB;
+    const bool tail_pair = (t_end - last_b * KB < KB) && (last_b * KB >= t_begin) &&
+                           owner_of((last_b + 1) * KB - 1, p.T, p.G) == cta + 1;
+    float pre[MT][4];
+    bool have_pre = false;
 
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t fix_phase = 0;
-    const int64_t first_b = t_begin / p.KB;
-    int64_t seg_start = t_begin;
+    uint32_t b = first_b;                       // channel block of tile t
+    uint32_t kb = t_begin - first_b * KB;       // its K block
+    bool seg_whole = (kb == 0);                 // segment started at K block 0
+    bool seg_new = true;
 
-    for (int64_t t = t_begin; t < t_end;) {
-        const int64_t b = t / p.KB;
-        const int kb = (int)(t % p.KB);
-        const int cnt = (int)min64(kTilesPerStage, min64(t_end - t, p.KB - kb));
+    for (uint32_t t = t_begin; t < t_end;) {
+        if (seg_new) {
+            seg_new = false;
+            if (tail_pair && b == last_b) {
+                if (threadIdx.x == 0) last_flag[0] = (ld_acquire_gpu(&p.counters[b]) == 1);
+                if (!consumers_sync()) return;
+                have_pre = last_flag[0] != 0;
+                if (have_pre) {
+                    const float *src = p.partials + (int64_t)(2 * (cta + 1)) * C::kPartialFloats;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            pre[mt][e] = __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
+                }
+            }
+        }
+        const int cnt = (int)min(min((uint32_t)kTilesPerStage, t_end - t), KB - kb);
         if (!mbar_wait(&full[stage], phase, SITE_DEC_FULL)) return;
         const uint8_t *ws = base + stage * C::kStageBytes;
         const uint8_t *xs = ws + kStageW;
-        for (int j = 0; j < cnt; ++j) {
-            const uint8_t *tile = ws + j * kTileBytes;
-            const uint4 alo = *reinterpret_cast<const uint4 *>(tile + a_off_lo);
-            const uint4 ahi = *reinterpret_cast<const uint4 *>(tile + a_off_hi);
-            uint4 xv[MT][2];
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                xv[mt][0] = *reinterpret_cast<const uint4 *>(xs + j * C::kXBoxBytes + x_off[mt][0]);
-                xv[mt][1] = *reinterpret_cast<const uint4 *>(xs + j * C::kXBoxBytes + x_off[mt][1]);
-            }
-            const uint32_t wl[4] = {alo.x, alo.y, alo.z, alo.w};
-            const uint32_t wh[4] = {ahi.x, ahi.y, ahi.z, ahi.w};
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t a0 = unbias2(widen_lo2(wl[jj]));   // row g,   k +0,+1
-                const uint32_t a1 = unbias2(widen_lo2(wh[jj]));   // row g+8, k +0,+1
-                const uint32_t a2 = unbias2(widen_hi2(wl[jj]));   // row g,   k +2,+3
-                const uint32_t a3 = unbias2(widen_hi2(wh[jj]));   // row g+8, k +2,+3
+        for (int j = 0; j < kTilesPerStage; ++j) {
+            if (j < cnt) {
+                const uint8_t *tile = ws + j * kTileBytes;
+                const uint4 alo = *reinterpret_cast<const uint4 *>(tile + a_off_lo);
+                const uint4 ahi = *reinterpret_cast<const uint4 *>(tile + a_off_hi);
+                uint4 xv[MT][2];
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
-                    const uint4 &xq = xv[mt][jj >> 1];
-                    const uint32_t b0 = (jj & 1) ? xq.z : xq.x;
-                    const uint32_t b1 = (jj & 1) ? xq.w : xq.y;
-                    mma_16816(acc[mt], a0, a1, a2, a3, b0, b1);
+                    xv[mt][0] = *reinterpret_cast<const uint4 *>(xs + j * C::kXBoxBytes + x_off[mt][0]);
+                    xv[mt][1] = *reinterpret_cast<const uint4 *>(xs + j * C::kXBoxBytes + x_off[mt][1]);
+                }
+                const uint32_t wl[4] = {alo.x, alo.y, alo.z, alo.w};
+                const uint32_t wh[4] = {ahi.x, ahi.y, ahi.z, ahi.w};
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t a0 = unbias2(widen_lo2(wl[jj]));   // row g,   k +0,+1
+                    const uint32_t a1 = unbias2(widen_lo2(wh[jj]));   // row g+8, k +0,+1
+                    const uint32_t a2 = unbias2(widen_hi2(wl[jj]));   // row g,   k +2,+3
+                    const uint32_t a3 = unbias2(widen_hi2(wh[jj]));   // row g+8, k +2,+3
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const uint4 &xq = xv[mt][jj >> 1];
+                        const uint32_t b0 = (jj & 1) ? xq.z : xq.x;
+                        const uint32_t b1 = (jj & 1) ? xq.w : xq.y;
+                        mma_16816(acc[mt][jj], a0, a1, a2, a3, b0, b1);
+                    }
                 }
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
         t += cnt;
+        kb += cnt;
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (t != t_end && kb != KB) continue;
 
-        if (t == t_end || t % p.KB == 0) {
-            // segment [seg_start, t) of channel block b is complete
-            const bool whole = (seg_start % p.KB == 0) && (t - seg_start == p.KB);
-            if (whole) {
-                store_y<MT>(p, b, warp, lane, acc);
-            } else {
-                const int slot = (b == first_b) ? 2 * cta : 2 * cta + 1;
-                float *mine = p.partials + (int64_t)slot * C::kPartialFloats;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        mine[(warp * 4 * MT + 4 * mt + e) * 32 + lane] = acc[mt][e];
-                __threadfence();
-                mbar_arrive(&fix_bar);
-                if (!mbar_wait(&fix_bar, fix_phase, SITE_DEC_FULL)) return;
-                fix_phase ^= 1u;
-                const int j_first = owner_of(b * p.KB, p.T, p.G);
-                const int j_last = owner_of((b + 1) * p.KB - 1, p.T, p.G);
-                if (threadIdx.x == 0) {
-                    const int old = atomicAdd(&p.counters[b], 1);
-                    last_flag = (old == j_last - j_first);
-                }
-                mbar_arrive(&fix_bar);
-                if (!mbar_wait(&fix_bar, fix_phase, SITE_DEC_FULL)) return;
-                fix_phase ^= 1u;
-                if (last_flag) {
-                    __threadfence();
-                    float sum[MT][4];
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) sum[mt][e] = 0.0f;
-                    for (int j = j_first; j <= j_last; ++j) {
-                        const int sj = (range_start(j, p.T, p.G) / p.KB == b) ? 2 * j : 2 * j + 1;
-                        const float *src = p.partials + (int64_t)sj * C::kPartialFloats;
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                sum[mt][e] += __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
-                    }
-                    store_y<MT>(p, b, warp, lane, sum);
-                    if (threadIdx.x == 0) p.counters[b] = 0;
-                }
-            }
+        // ------------------------------------------------ end of a segment
+        // This CTA's part of channel block b is done.  It is the whole block
+        // if it started at K block 0 and reached the end.
+        float sum[MT][4];
+        fold<MT>(acc, sum);
+        if (seg_whole && kb == KB) {
+            store_y<MT>(p, b, warp, lane, sum);
+        } else if (have_pre && b == last_b) {
+            // partner's part already in registers: own part first, then the
+            // partner's, the same order the general path uses
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc[mt][e] = 0.0f;
-            seg_start = t;
+                for (int e = 0; e < 4; ++e) sum[mt][e] += pre[mt][e];
+            store_y<MT>(p, b, warp, lane, sum);
+            if (threadIdx.x == 0) p.counters[b] = 0;
+        } else {
+            // publish this part; the last contributor to arrive adds all
+            // parts in CTA order (independent of arrival order), scales and
+            // stores, then resets the block's counter
+            const int slot = (b == first_b) ? 2 * cta : 2 * cta + 1;
+            float *mine = p.partials + (int64_t)slot * C::kPartialFloats;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    __stcg(&mine[(warp * 4 * MT + 4 * mt + e) * 32 + lane], sum[mt][e]);
+            if (!consumers_sync()) return;
+            const uint32_t j_first = owner_of(b * KB, p.T, p.G);
+            const uint32_t j_last = owner_of((b + 1) * KB - 1, p.T, p.G);
+            if (threadIdx.x == 0) {
+                __threadfence();   // with the barrier above: every thread's part
+                const int old = atomicAdd(&p.counters[b], 1);
+                last_flag[1] = ((uint32_t)old == j_last - j_first);
+            }
+            if (!consumers_sync()) return;
+            if (last_flag[1]) {
+                __threadfence();
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sum[mt][e] = 0.0f;
+                for (uint32_t j = j_first; j <= j_last; ++j) {
+                    const uint32_t sj = (range_start(j, p.T, p.G) / KB == b) ? 2 * j : 2 * j + 1;
+                    const float *src = p.partials + (int64_t)sj * C::kPartialFloats;
+                    float part[MT][4];
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            part[mt][e] = __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sum[mt][e] += part[mt][e];
+                }
+                store_y<MT>(p, b, warp, lane, sum);
+                if (threadIdx.x == 0) p.counters[b] = 0;
+            }
         }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[mt][jj][e] = 0.0f;
+        if (kb == KB) { kb = 0; ++b; }
+        seg_whole = true;
+        seg_new = true;
     }
 }
 

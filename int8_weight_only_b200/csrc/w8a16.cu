@@ -319,12 +319,29 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
         p.M = (int)M;
         p.N = N;
         p.KB = KB;
-        p.T = NB * KB;
-        p.G = decode_grid(d->sms, p.T);
-        if (MT == 1)
-            decode::decode_kernel<1><<<p.G, decode::kThreads, decode::Cfg<1>::kSmemBytes, st>>>(map, p);
-        else
-            decode::decode_kernel<2><<<p.G, decode::kThreads, decode::Cfg<2>::kSmemBytes, st>>>(map, p);
+        const int64_t T = NB * KB;
+        const int G = decode_grid(d->sms, T);
+        if ((uint64_t)T * (uint64_t)(G + 1) >= (1ull << 32)) return W8_ERR_SHAPE;
+        p.T = (uint32_t)T;
+        p.G = (uint32_t)G;
+        // programmatic dependent launch: this kernel's prologue and an L2
+        // prefetch of its first weight tiles overlap the previous kernel
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)G, 1, 1);
+        cfg.blockDim = dim3(decode::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = MT == 1 ? decode::Cfg<1>::kSmemBytes : decode::Cfg<2>::kSmemBytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = MT == 1 ? cudaLaunchKernelEx(&cfg, decode::decode_kernel<1>, map, p)
+                                      : cudaLaunchKernelEx(&cfg, decode::decode_kernel<2>, map, p);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return W8_ERR_CUDA;
+        }
         return launch_status();
     }
 
@@ -472,8 +489,11 @@ extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *pack
     p.M = (int)M;
     p.N = N;
     p.KB = KB;
-    p.T = NB * KB;
-    p.G = decode_grid(d->sms, p.T);
+    const int64_t T = NB * KB;
+    const int G = decode_grid(d->sms, T);
+    if ((uint64_t)T * (uint64_t)(G + 1) >= (1ull << 32)) return W8_ERR_LIMIT;
+    p.T = (uint32_t)T;
+    p.G = (uint32_t)G;
     if (MT == 1)
         decode::decode_kernel<1><<<p.G, decode::kThreads, decode::Cfg<1>::kSmemBytes, st>>>(map, p);
     else
