@@ -20,6 +20,9 @@ __device__ unsigned int g_status;
 
 enum WaitSite : unsigned {
     SITE_Q_LOAD = 0x10,
+    SITE_Q_EMPTY = 0x11,
+    SITE_Q_XCHG = 0x12,
+    SITE_Q_SYNC = 0x13,
     SITE_DEC_EMPTY = 0x20,
     SITE_DEC_FULL = 0x21,
     SITE_DEC_FIX = 0x22,
@@ -120,6 +123,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
     return ok != 0;
 }
 
+// try_wait that may park the thread (without issuing) for up to `hint_ns`
+// until the phase completes, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar_addr, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for waiters that should not take issue slots from the
+// threads doing the work (many warps waiting on one barrier): each try
+// parks the thread for up to 20 us.
+__device__ __forceinline__ bool mbar_wait_parked(uint64_t *bar, uint32_t parity, unsigned site,
+                                                 unsigned long long limit_ns = kWaitLimitNs) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+#pragma unroll 1
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i) {
+            if (mbar_try_wait_sleep(a, parity, 20000u)) return true;
+        }
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_timeout(site);
+            return false;
+        }
+    }
+}
+
 // Wait until the barrier's phase with the given parity has completed.
 // Gives up after `limit_ns`, records `site` and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned site,
@@ -144,6 +182,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
         }
     }
 }
+
+// The same decision in every lane of the warp (all lanes must call it):
+// after a bounded wait, lanes whose waits ended differently would otherwise
+// diverge before warp-collective instructions.
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok) != 0; }
 
 // ---------------------------------------------------------------- TMA
 // 1-D bulk copy global -> shared, completion counted on `bar` in bytes.
@@ -185,8 +228,91 @@ __device__ __forceinline__ void tma_load_2d(void *dst_smem, const CUtensorMap *m
         : "memory");
 }
 
+// Same with an L2 eviction-priority policy (createpolicy result).
+__device__ __forceinline__ void tma_load_2d_hint(void *dst_smem, const CUtensorMap *map, int32_t x,
+                                                 int32_t y, uint64_t *bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+// Arrive once on an mbarrier of some CTA of the cluster, releasing this
+// thread's prior writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar_addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait on a local barrier whose arrivals come from the whole
+// cluster (acquire at cluster scope).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, unsigned site,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
+    const uint32_t a = smem_u32(bar);
+#pragma unroll 1
+    for (int i = 0; i < 512; ++i) {
+        if (mbar_try_wait_acq_cluster(a, parity)) return true;
+    }
+    const unsigned long long t0 = globaltimer_ns();
+#pragma unroll 1
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 512; ++i) {
+            if (mbar_try_wait_acq_cluster(a, parity)) return true;
+        }
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_timeout(site);
+            return false;
+        }
+    }
+}
+// Full cluster barrier (every thread of every CTA of the cluster).
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
 }
 
 // ---------------------------------------------------------------- named barriers

@@ -5,14 +5,25 @@
 //   q[k,n] = clamp( rne( W[k,n] / float(s_n) ), -127, 127 ),  q = 0 if s_n == 0
 //
 // HBM-bound: the algorithmic traffic is one read of W (4 or 2 bytes per
-// weight) plus one write of q (1 byte per weight).  To read W only once,
-// a thread-block cluster of CQ CTAs owns a strip of BN columns: CTA r of the
-// cluster stages rows [r*kc, (r+1)*kc) of the strip in shared memory with
-// 2-D TMA loads, reduces its per-column |max|, the cluster combines the CQ
-// partial maxima through distributed shared memory, and every CTA then
-// quantizes its rows straight from shared memory.  When K is too large for
-// the strip to stay resident (K * BN * elem > cluster shared memory), the
-// same kernel streams the rows twice (max pass, then quantize pass).
+// weight) plus one write of q (1 byte per weight).  Design:
+//  - Work unit: a panel of 32 columns over all K rows.  A thread-block
+//    cluster of C CTAs owns a panel; CTA r of the cluster takes rows
+//    [r kc, (r+1) kc).  Clusters are persistent (as many as fit at once)
+//    and walk the panels.
+//  - One producer thread per CTA streams each panel's rows twice through
+//    one 4-stage shared-memory ring (two CTAs per SM) with 2-D TMA loads: pass 1 (L2
+//    evict-last) for the column |max|, pass 2 (evict-first) to quantize.
+//    The passes are interleaved one panel apart -- P1(0) P1(1) P2(0) P1(2)
+//    P2(1) ... -- so pass 1 of the next panel streams from HBM while this
+//    panel's maxima are combined, and pass 2 reads L2: the rows held between
+//    the passes are two slices per CTA, a few tens of MB in all.
+//  - The C partial maxima of a panel are combined over distributed shared
+//    memory: each CTA publishes its 32 partial maxima, arrives on every
+//    peer's exchange barrier, and before pass 2 reads all peers' values.
+//  - q = rne(w / s) is computed as rne(w * fl(1/s)) where that product is
+//    provably on the same side of every rounding boundary as the correctly
+//    rounded quotient, and with the IEEE division otherwise (see
+//    quantize_fast), so the codes are those of the exact definition.
 #pragma once
 
 #include "common.cuh"
@@ -20,178 +31,317 @@
 namespace w8 {
 namespace quant {
 
-constexpr int kThreads = 256;
-constexpr int kBoxRows = 64;          // rows per TMA box
-constexpr int kMaxBoxes = 32;         // mbarriers per CTA
+constexpr int kConsumerWarps = 16;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;
+constexpr int kPanel = 32;          // columns per panel
+constexpr int kStages = 4;
+constexpr int kBoxBytes = 16384;    // one ring slot
+constexpr int kSmemBytes = kStages * kBoxBytes + 1024;
+constexpr int kMaxCluster = 8;
+constexpr int kPartBufs = 3;        // partial-maxima buffers (see the exchange)
 
+// Box geometry: 128 fp32 rows or 256 fp16 rows of 32 columns (16 KB).  A
+// consumer thread owns one 16-byte segment of a row: 4 fp32 or 8 fp16
+// columns; kThreadsPerRow threads cover a row, kSweep rows per sweep of all
+// consumers, kSweeps sweeps per box.
 template <typename T>
-__device__ __forceinline__ float to_f32(T v);
-template <>
-__device__ __forceinline__ float to_f32<float>(float v) { return v; }
-template <>
-__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+struct Box {
+    static constexpr int kCols = 16 / (int)sizeof(T);
+    static constexpr int kThreadsPerRow = kPanel / kCols;
+    static constexpr int kRowBytes = kPanel * (int)sizeof(T);
+    static constexpr int kRows = kBoxBytes / kRowBytes;
+    static constexpr int kSweep = kConsumers / kThreadsPerRow;
+    static constexpr int kSweeps = kRows / kSweep;
+};
 
-// 4 consecutive elements of one row, widened to fp32.
-template <typename T>
-__device__ __forceinline__ void load4(const T *p, float (&v)[4]);
-template <>
-__device__ __forceinline__ void load4<float>(const float *p, float (&v)[4]) {
-    float4 t = *reinterpret_cast<const float4 *>(p);
-    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+// rne(w / s) clamped to [-127, 127], equal to the correctly rounded quotient
+// rounded to the nearest integer (ties to even), with inv_s = fl(1/s).
+//
+// r = fl(w * inv_s) differs from the exact w/s by at most 2^-23 |w/s|
+// (two roundings of relative size 2^-24), and the correctly rounded
+// quotient fl(w/s) differs from w/s by at most 2^-24 |w/s|.  For |r| < 126
+// both are within 2^-15 of each other, so when r is more than 2^-13 away
+// from every half-integer both round to the same integer (and no clamp
+// applies).  Otherwise the quotient is formed with the IEEE division.
+//
+// Split in two so a row segment takes one branch, not one per element:
+// quantize_fast returns rne(r) and whether r was unambiguous; for s == 0
+// the caller passes inv_s = 0, so r = 0 and the code is 0 as defined.
+// It stays off the special-function unit (no floor, no float-to-int
+// conversion): adding 1.5 * 2^23 rounds |r| < 2^22 to the nearest integer,
+// ties to even (the sum's unit in the last place is 1), and that integer
+// is the sum's low mantissa bits, i.e. its bit pattern minus 0x4B400000.
+// The distance from r to the nearest integer then decides whether r is
+// more than 2^-13 away from every half-integer.
+__device__ __forceinline__ int quantize_fast(float w, float inv_s, bool &sure) {
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+    const float r = w * inv_s;
+    const float t = r + kMagic;
+    const float d = fabsf(r - (t - kMagic));
+    sure = (fabsf(r) < 126.0f) & (d < 0.5f - 0x1p-13f);
+    return __float_as_int(t) - 0x4B400000;
 }
-template <>
-__device__ __forceinline__ void load4<__half>(const __half *p, float (&v)[4]) {
-    uint2 t = *reinterpret_cast<const uint2 *>(p);
-    __half2 a = *reinterpret_cast<__half2 *>(&t.x);
-    __half2 b = *reinterpret_cast<__half2 *>(&t.y);
-    v[0] = __low2float(a); v[1] = __high2float(a);
-    v[2] = __low2float(b); v[3] = __high2float(b);
-}
-
-__device__ __forceinline__ int quantize_one(float w, float s) {
+__device__ __forceinline__ int quantize_exact(float w, float s) {
     if (s == 0.0f) return 0;
-    int v = __float2int_rn(__fdiv_rn(w, s));   // IEEE division, ties to even
+    const int v = __float2int_rn(__fdiv_rn(w, s));
     return max(-127, min(127, v));
 }
 
-// Launch: grid.x = CQ * ceil(N / BN) with cluster dims (CQ, 1, 1); the
-// cluster rank is the K slice.  Dynamic shared memory: nbuf boxes of
-// kBoxRows x BN elements plus 1 KB of alignment slack.
-//   kc      rows per CTA (multiple of kBoxRows)
-//   nbuf    boxes held in shared memory (== kc / kBoxRows when resident)
-template <typename T, int BN>
-__global__ void __launch_bounds__(kThreads)
-quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, int64_t K, int64_t N, int kc,
-                int nbuf, int8_t *__restrict__ q, uint16_t *__restrict__ scales) {
-    static_assert(BN % 4 == 0 && (kThreads / (BN / 4)) * (BN / 4) == kThreads, "layout");
-    constexpr int kColGroups = BN / 4;                  // threads per row
-    constexpr int kRowsPerPass = kThreads / kColGroups; // rows per sweep
-    constexpr int kBoxElems = kBoxRows * BN;
-    constexpr uint32_t kBoxBytes = kBoxElems * sizeof(T);
+// The 16-byte row segment of a thread, widened to fp32.
+template <typename T>
+__device__ __forceinline__ void load_seg(const uint8_t *p, float (&v)[Box<T>::kCols]);
+template <>
+__device__ __forceinline__ void load_seg<float>(const uint8_t *p, float (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void load_seg<__half>(const uint8_t *p, float (&v)[8]) {
+    const uint4 a = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
+        v[2 * i] = __low2float(h);
+        v[2 * i + 1] = __high2float(h);
+    }
+}
 
+struct Params {
+    int8_t *q;
+    uint16_t *scales;
+    int64_t K;
+    int64_t N;
+    int kc;            // rows per cluster rank (multiple of the box height)
+    int panels;        // ceil(N / 32)
+    int clusters;      // clusters in the grid
+};
+
+// grid = clusters * C CTAs, cluster dims (C, 1, 1), kThreads threads,
+// kSmemBytes dynamic shared memory.  The tensor map covers W [K, N] with
+// a box of 32 columns x Box<T>::kRows rows, no swizzle.
+//
+// Step j of a CTA (panels P_j = cid + j * clusters):
+//   (a) pass 1 over P_j, partial maxima into part[j % 3];
+//   (b) wait until every peer published P_{j-1}, read the peers' partial
+//       maxima of P_{j-1}, form its scales;
+//   (c) arrive on every peer's exchange barrier for P_j (this also tells
+//       the peers that P_{j-1}'s values have been read here);
+//   (d) pass 2 over P_{j-1}.
+// A CTA overwrites part[j % 3] in (a) only after its own (b) of step j-1,
+// which waited for the peers' (c) of step j-1, issued after their reads of
+// P_{j-2} -- the values part[j % 3] held before -- so three buffers never
+// race.  The exchange barriers alternate by panel parity.
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2)
+quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
+    using B = Box<T>;
     extern __shared__ uint8_t smem_raw[];
-    T *buf = reinterpret_cast<T *>(
+    uint8_t *ring = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t bars[kMaxBoxes];
-    __shared__ float red[kRowsPerPass][BN + 1];
-    __shared__ float cta_amax[BN];
-    __shared__ float col_scale[BN];
-    __shared__ int abort_flag;
+    __shared__ uint64_t full[kStages], empty[kStages];
+    __shared__ uint64_t xbar[2];                    // exchange barriers, by panel parity
+    __shared__ uint64_t cbar;                       // consumer-only barrier
+    __shared__ float part[kPartBufs][kPanel];       // this CTA's partial maxima
+    __shared__ float red[kConsumerWarps][kPanel];
+    __shared__ float col_scale[kPanel];
+    __shared__ float col_inv[kPanel];
 
-    uint32_t rank;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
-    uint32_t csize;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(csize));
-    const int64_t strip = blockIdx.x / csize;
-    const int64_t n0 = strip * BN;
-    const int64_t k_begin = (int64_t)rank * kc;
-    const int64_t k_end = min64(K, k_begin + (int64_t)kc);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const uint32_t csize = cluster_size();
+    const int cid = blockIdx.x / csize;
+    const int64_t k_begin = (int64_t)rank * p.kc;
+    const int64_t k_end = min64(p.K, k_begin + p.kc);
     const int rows = (int)max64(0, k_end - k_begin);
-    const int nbox = (rows + kBoxRows - 1) / kBoxRows;
-    const bool resident = nbox <= nbuf;
-    const int tid = threadIdx.x;
-    const int cg = tid % kColGroups;     // column group: columns 4cg .. 4cg+3
-    const int rg = tid / kColGroups;     // row within a sweep
+    const int nbox = (rows + B::kRows - 1) / B::kRows;
+    const int npan = cid < p.panels ? (p.panels - cid + p.clusters - 1) / p.clusters : 0;
 
-    if (tid == 0) {
-        abort_flag = 0;
-        for (int i = 0; i < nbuf; ++i) mbar_init(&bars[i], 1);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kConsumerWarps);
+        }
+        mbar_init(&xbar[0], csize);
+        mbar_init(&xbar[1], csize);
+        mbar_init(&cbar, kConsumers);
         fence_barrier_init();
         prefetch_tensormap(&tmap_w);
     }
-    __syncthreads();
+    // barrier initialisation is visible to the whole cluster before any
+    // remote arrive
+    cluster_sync_all();
 
-    uint32_t phase_bits = 0;   // bit i: parity of the next completion of bars[i]
-
-    // Issue box `i` into buffer slot i % nbuf (thread 0 only).
-    auto issue = [&](int i) {
-        const int slot = i % nbuf;
-        mbar_arrive_expect_tx(&bars[slot], kBoxBytes);
-        tma_load_2d(buf + (size_t)slot * kBoxElems, &tmap_w, (int32_t)n0,
-                    (int32_t)(k_begin + (int64_t)i * kBoxRows), &bars[slot]);
-    };
-    auto wait_box = [&](int i) -> bool {
-        const int slot = i % nbuf;
-        const bool ok = mbar_wait(&bars[slot], (phase_bits >> slot) & 1u, SITE_Q_LOAD);
-        phase_bits ^= 1u << slot;
-        return ok;
-    };
-
-    // ---------------- pass 1: per-column |max| over this CTA's rows
-    float amax[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int g0 = 0; g0 < nbox; g0 += nbuf) {
-        const int g1 = min(nbox, g0 + nbuf);
-        if (tid == 0)
-            for (int i = g0; i < g1; ++i) issue(i);
-        for (int i = g0; i < g1; ++i) {
-            if (!wait_box(i)) abort_flag = 1;
-            const T *box = buf + (size_t)(i % nbuf) * kBoxElems;
-            const int box_rows = min(kBoxRows, rows - i * kBoxRows);
-            for (int r = rg; r < box_rows; r += kRowsPerPass) {
-                float v[4];
-                load4<T>(box + r * BN + 4 * cg, v);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) amax[j] = fmaxf(amax[j], fabsf(v[j]));
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+            int s = 0;
+            uint32_t ph = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int j = 0; j <= npan && ok; ++j) {
+                for (int pass = 0; pass < 2 && ok; ++pass) {
+                    // pass 0: P1 of panel j; pass 1: P2 of panel j - 1
+                    const int pj = pass == 0 ? j : j - 1;
+                    if (pj < 0 || pj >= npan) continue;
+                    const int panel = cid + pj * p.clusters;
+                    for (int i = 0; i < nbox; ++i) {
+                        if (!mbar_wait_parked(&empty[s], ph ^ 1u, SITE_Q_EMPTY)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&full[s], kBoxBytes);
+                        tma_load_2d_hint(ring + s * kBoxBytes, &tmap_w, panel * kPanel,
+                                         (int32_t)(k_begin + (int64_t)i * B::kRows), &full[s],
+                                         pass == 0 ? keep : drop);
+                        ++issued;
+                        if (++s == kStages) { s = 0; ph ^= 1u; }
+                    }
+                }
+            }
+            // every issued copy has landed before the CTA can leave
+            for (int i = 0; i < kStages && i < issued; ++i) {
+                if (--s < 0) { s = kStages - 1; ph ^= 1u; }
+                mbar_wait(&full[s], ph, SITE_Q_LOAD, 10000000ull);
             }
         }
-        if (!resident) __syncthreads();   // slots are reused by the next group
-    }
+    } else {
+        // ------------------------------------------------------ consumers
+        const int c = threadIdx.x;                  // 0 .. kConsumers - 1
+        const int t = c % B::kThreadsPerRow;        // column segment
+        const int rsub = c / B::kThreadsPerRow;     // row within a sweep
+        const int col0 = t * B::kCols;              // first panel column of the segment
+        int s = 0;
+        uint32_t ph = 0;
+        uint32_t cph = 0;
+        bool ok = true;
+        auto csync = [&]() -> bool {
+            mbar_arrive(&cbar);
+            const bool r = warp_all(mbar_wait_parked(&cbar, cph, SITE_Q_SYNC));
+            cph ^= 1u;
+            return r;
+        };
+        for (int j = 0; j <= npan && ok; ++j) {
+            // ---------------- (a) pass 1 over panel j: column |max|
+            if (j < npan) {
+                float amax[B::kCols];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) red[rg][4 * cg + j] = amax[j];
-    __syncthreads();
-    if (tid < BN) {
-        float m = 0.f;
-        for (int r = 0; r < kRowsPerPass; ++r) m = fmaxf(m, red[r][tid]);
-        cta_amax[tid] = m;
-    }
-    // ---------------- cluster-wide maximum through distributed shared memory
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    if (tid < BN) {
-        float m = 0.f;
-        const uint32_t local = smem_u32(&cta_amax[tid]);
-        for (uint32_t r = 0; r < csize; ++r) {
-            uint32_t remote;
-            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(r));
-            float v;
-            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-            m = fmaxf(m, v);
-        }
-        const __half s16 = __float2half_rn(__fdiv_rn(m, 127.0f));
-        col_scale[tid] = __half2float(s16);
-        if (rank == 0 && n0 + tid < N) scales[n0 + tid] = __half_as_ushort(s16);
-    }
-    // no CTA may leave while a peer still reads its cta_amax
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-
-    // ---------------- pass 2: quantize (from shared memory when resident)
-    float s[4];
+                for (int e = 0; e < B::kCols; ++e) amax[e] = 0.0f;
+                for (int i = 0; i < nbox; ++i) {
+                    if (!warp_all(mbar_wait_parked(&full[s], ph, SITE_Q_LOAD))) { ok = false; break; }
+                    const uint8_t *box = ring + s * kBoxBytes;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) s[j] = col_scale[4 * cg + j];
-    const bool col_ok = (n0 + 4 * cg) < N;   // N % 8 == 0: groups of 4 are all in or all out
-    for (int g0 = 0; g0 < nbox; g0 += nbuf) {
-        const int g1 = min(nbox, g0 + nbuf);
-        if (!resident) {
-            if (tid == 0)
-                for (int i = g0; i < g1; ++i) issue(i);
-        }
-        for (int i = g0; i < g1; ++i) {
-            if (!resident && !wait_box(i)) abort_flag = 1;
-            const T *box = buf + (size_t)(i % nbuf) * kBoxElems;
-            const int box_rows = min(kBoxRows, rows - i * kBoxRows);
-            for (int r = rg; r < box_rows; r += kRowsPerPass) {
-                float v[4];
-                load4<T>(box + r * BN + 4 * cg, v);
-                uint32_t packed = 0;
+                    for (int w = 0; w < B::kSweeps; ++w) {
+                        float v[B::kCols];
+                        load_seg<T>(box + (rsub + w * B::kSweep) * B::kRowBytes + 16 * t, v);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    packed |= (uint32_t)(quantize_one(v[j], s[j]) & 0xFF) << (8 * j);
-                const int64_t k = k_begin + (int64_t)i * kBoxRows + r;
-                if (col_ok)
-                    *reinterpret_cast<uint32_t *>(q + k * N + n0 + 4 * cg) = packed;
+                        for (int e = 0; e < B::kCols; ++e) amax[e] = fmaxf(amax[e], fabsf(v[e]));
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);
+                    if (++s == kStages) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                // lanes with the same t hold the same columns
+#pragma unroll
+                for (int off = B::kThreadsPerRow; off < 32; off <<= 1)
+#pragma unroll
+                    for (int e = 0; e < B::kCols; ++e)
+                        amax[e] = fmaxf(amax[e], __shfl_xor_sync(0xffffffffu, amax[e], off));
+                if (lane < B::kThreadsPerRow) {
+#pragma unroll
+                    for (int e = 0; e < B::kCols; ++e) red[warp][col0 + e] = amax[e];
+                }
+                if (!csync()) { ok = false; break; }
+                if (c < kPanel) {
+                    float m = 0.0f;
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) m = fmaxf(m, red[w][c]);
+                    part[j % kPartBufs][c] = m;
+                }
+            }
+            if (j == 0) {
+                // (c) for panel 0; nothing to read yet
+                if (!csync()) { ok = false; break; }
+                if (c < (int)csize) mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[0]), (uint32_t)c));
+                continue;
+            }
+            // ---------------- (b) combine the maxima of panel j - 1
+            const int pj = j - 1;
+            const int panel = cid + pj * p.clusters;
+            if (!warp_all(mbar_wait_cluster(&xbar[pj & 1], (pj >> 1) & 1, SITE_Q_XCHG))) { ok = false; break; }
+            if (c < kPanel) {
+                float m = 0.0f;
+                const uint32_t local = smem_u32(&part[pj % kPartBufs][c]);
+                for (uint32_t r = 0; r < csize; ++r) m = fmaxf(m, ld_dsmem_f32(mapa_shared(local, r)));
+                const __half s16 = __float2half_rn(__fdiv_rn(m, 127.0f));
+                const float sf = __half2float(s16);
+                col_scale[c] = sf;
+                col_inv[c] = sf != 0.0f ? __frcp_rn(sf) : 0.0f;
+                const int64_t n = (int64_t)panel * kPanel + c;
+                if (rank == 0 && n < p.N) p.scales[n] = __half_as_ushort(s16);
+            }
+            // every consumer's partial maxima of panel j are in part[] and
+            // every read of panel j - 1's values is done
+            if (!csync()) { ok = false; break; }
+            // ---------------- (c) publish panel j
+            if (j < npan && c < (int)csize)
+                mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[j & 1]), (uint32_t)c));
+            // ---------------- (d) pass 2 over panel j - 1 (from L2)
+            float sc[B::kCols], inv[B::kCols];
+#pragma unroll
+            for (int e = 0; e < B::kCols; ++e) {
+                sc[e] = col_scale[col0 + e];
+                inv[e] = col_inv[col0 + e];
+            }
+            const int64_t n0 = (int64_t)panel * kPanel + col0;
+            const bool cols_ok = n0 < p.N;   // N % 8 == 0: a segment is all in or all out
+            for (int i = 0; i < nbox; ++i) {
+                if (!warp_all(mbar_wait_parked(&full[s], ph, SITE_Q_LOAD))) { ok = false; break; }
+                const uint8_t *box = ring + s * kBoxBytes;
+#pragma unroll
+                for (int w = 0; w < B::kSweeps; ++w) {
+                    const int rloc = rsub + w * B::kSweep;
+                    float v[B::kCols];
+                    load_seg<T>(box + rloc * B::kRowBytes + 16 * t, v);
+                    int code[B::kCols];
+                    bool sure = true;
+#pragma unroll
+                    for (int e = 0; e < B::kCols; ++e) {
+                        bool se;
+                        code[e] = quantize_fast(v[e], inv[e], se);
+                        sure &= se;
+                    }
+                    if (!sure) {   // rare: some product lies near a rounding boundary
+#pragma unroll
+                        for (int e = 0; e < B::kCols; ++e) code[e] = quantize_exact(v[e], sc[e]);
+                    }
+                    uint32_t packed[B::kCols / 4];
+#pragma unroll
+                    for (int g = 0; g < B::kCols / 4; ++g) {
+                        // low bytes of four codes into one word
+                        const uint32_t lo = __byte_perm((uint32_t)code[4 * g], (uint32_t)code[4 * g + 1], 0x0040);
+                        const uint32_t hi = __byte_perm((uint32_t)code[4 * g + 2], (uint32_t)code[4 * g + 3], 0x0040);
+                        packed[g] = __byte_perm(lo, hi, 0x5410);
+                    }
+                    const int64_t k = k_begin + (int64_t)i * B::kRows + rloc;
+                    if (k < k_end && cols_ok) {
+                        int8_t *dst = p.q + k * p.N + n0;
+                        if (B::kCols == 4)
+                            *reinterpret_cast<uint32_t *>(dst) = packed[0];
+                        else
+                            *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[B::kCols / 4 - 1]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                if (++s == kStages) { s = 0; ph ^= 1u; }
             }
         }
-        if (!resident) __syncthreads();
     }
+    // no CTA leaves while a peer may still read its shared memory or arrive
+    // on its barriers; every thread reaches this point on every path
+    cluster_sync_all();
 }
 
 }  // namespace quant

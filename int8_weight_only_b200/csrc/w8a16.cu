@@ -26,6 +26,9 @@ struct DeviceInfo {
     bool ready = false;
     int status = W8_OK;   // W8_ERR_DEVICE if not sm_100
     int sms = 0;
+    // resident quantize clusters per cluster size (0 = not yet queried)
+    int qclusters_f32[quant::kMaxCluster + 1] = {};
+    int qclusters_f16[quant::kMaxCluster + 1] = {};
 };
 
 std::mutex g_mu;
@@ -57,16 +60,12 @@ int device_info(DeviceInfo **out) {
                 e = cudaFuncSetAttribute(prefill::prefill_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          prefill::kSmemBytes);
-            const int qmax = 201 * 1024;
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(quant::quantize_kernel<float, 32>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, qmax);
+                e = cudaFuncSetAttribute(quant::quantize_kernel<float>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, quant::kSmemBytes);
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(quant::quantize_kernel<float, 16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, qmax);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(quant::quantize_kernel<__half, 32>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, qmax);
+                e = cudaFuncSetAttribute(quant::quantize_kernel<__half>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, quant::kSmemBytes);
             if (e != cudaSuccess) return W8_ERR_CUDA;
         }
         d.ready = true;
@@ -117,40 +116,67 @@ inline int launch_status() {
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ---------------------------------------------------------------- quantize
-template <typename T, int BN>
-int launch_quantize(const void *W, CUtensorMapDataType dt, int64_t K, int64_t N, int8_t *q,
-                    uint16_t *scales, cudaStream_t st) {
-    constexpr int elem = sizeof(T);
-    constexpr int box_bytes = quant::kBoxRows * BN * elem;
-    constexpr int64_t target_rows = (64 * 1024) / (BN * elem);   // ~64 KB per CTA
-    constexpr int64_t resident_max = (200 * 1024) / box_bytes;  // boxes
-    int cq = (int)std::min<int64_t>(8, std::max<int64_t>(1, cdiv(K, target_rows)));
-    int64_t kc = cdiv(cdiv(K, cq), quant::kBoxRows) * quant::kBoxRows;
-    int64_t nbox = kc / quant::kBoxRows;
-    int nbuf = (int)std::min<int64_t>({nbox, resident_max, (int64_t)quant::kMaxBoxes});
-    if (nbox > nbuf) nbuf = (int)std::min<int64_t>(8, nbuf);   // streaming: 8 boxes in flight
-    if (kc > INT32_MAX) return W8_ERR_SHAPE;
+// Cluster size for K rows: the K range is split C ways so that the rows all
+// CTAs hold between their two passes (two slices of K/C rows x 128 B per
+// SM) stay well inside L2, so that small matrices still spread over the
+// SMs, and -- clusters of 8 leave a sixth of the SMs idle on this part --
+// preferring 4 where that suffices.
+inline int quantize_cluster(int64_t K, int rows_per_box) {
+    if (K > 8192) return quant::kMaxCluster;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(4, cdiv(K, 2 * rows_per_box)));
+}
+
+template <typename T>
+int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_t K, int64_t N,
+                    int8_t *q, uint16_t *scales, cudaStream_t st) {
+    constexpr int rows = quant::Box<T>::kRows;
+    const int C = quantize_cluster(K, rows);
+    const int64_t kc = cdiv(cdiv(K, C), rows) * rows;
+    const int64_t panels = cdiv(N, quant::kPanel);
+    if (kc > INT32_MAX || panels > INT32_MAX) return W8_ERR_SHAPE;
 
     CUtensorMap map;
-    int rc = make_map_2d(&map, W, dt, elem, (uint64_t)N, (uint64_t)K, BN, quant::kBoxRows,
+    int rc = make_map_2d(&map, W, dt, (int)sizeof(T), (uint64_t)N, (uint64_t)K, quant::kPanel, rows,
                          CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc != W8_OK) return rc;
 
-    const int64_t strips = cdiv(N, BN);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(strips * cq), 1, 1);
     cfg.blockDim = dim3(quant::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)nbuf * box_bytes + 1024;
+    cfg.dynamicSmemBytes = quant::kSmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cq;
+    attr[0].val.clusterDim.x = C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T, BN>, map, K, N, (int)kc, nbuf, q, scales) !=
-        cudaSuccess) {
+    // persistent clusters: as many as can be resident at once
+    int resident = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int &cached = sizeof(T) == 4 ? d->qclusters_f32[C] : d->qclusters_f16[C];
+        if (cached == 0) {
+            cfg.gridDim = dim3((unsigned)(C * d->sms), 1, 1);
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, quant::quantize_kernel<T>, &cfg) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                n = std::max(1, d->sms / C);
+            }
+            cached = n;
+        }
+        resident = cached;
+    }
+    quant::Params p;
+    p.q = q;
+    p.scales = scales;
+    p.K = K;
+    p.N = N;
+    p.kc = (int)kc;
+    p.panels = (int)panels;
+    p.clusters = (int)std::min<int64_t>(panels, resident);
+    cfg.gridDim = dim3((unsigned)(p.clusters * C), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T>, map, p) != cudaSuccess) {
         cudaGetLastError();
         return W8_ERR_CUDA;
     }
@@ -199,15 +225,9 @@ int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, in
     int rc = device_info(&d);
     if (rc != W8_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (w_dtype == W8_F32) {
-        // keep each CTA's strip resident in shared memory: 32 columns while
-        // it fits the cluster, else 16 (64-byte rows), else stream twice
-        const int64_t per_cta32 = cdiv(cdiv(K, 8), 64) * 64 * 32 * 4;
-        if (per_cta32 <= 112 * 1024 || cdiv(cdiv(K, 8), 64) * 64 * 16 * 4 > 200 * 1024)
-            return launch_quantize<float, 32>(W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, st);
-        return launch_quantize<float, 16>(W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, st);
-    }
-    return launch_quantize<__half, 32>(W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, st);
+    if (w_dtype == W8_F32)
+        return launch_quantize<float>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, st);
+    return launch_quantize<__half>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, st);
 }
 
 size_t w8_prepacked_bytes(int64_t K, int64_t N) {
