@@ -270,7 +270,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             }
         }
         const int cnt = (int)min(min((uint32_t)kTilesPerStage, t_end - t), KB - kb);
-        if (!mbar_wait(&full[stage], phase, SITE_DEC_FULL)) return;
+        // parked, not spinning: eight warps polling one barrier take issue
+        // slots from the warps that have data
+        if (!mbar_wait_parked(&full[stage], phase, SITE_DEC_FULL)) return;
         const uint8_t *ws = base + stage * C::kStageBytes;
         const uint8_t *xs = ws + kStageW;
 #pragma unroll

@@ -89,3 +89,27 @@ def test_quantize_bert_base_all_weights():
     for i, (K, N) in enumerate(synthetic.WORKLOADS["bert_base_4096_tokens"]["matrices"]):
         W = synthetic.weights(K, N, SEED, synthetic.tensor_id(5, 0, i, 0))
         _check(W)
+
+
+def test_quantize_near_rounding_boundaries():
+    # Each column's scale is an exact fp16 value s0 (its max is 127 * s0).
+    # The other weights sit at (k + 1/2 + d) * s0 for offsets d just inside
+    # and outside the band where a reciprocal-multiply and the correctly
+    # rounded quotient can disagree, and at exact ties; the codes must
+    # still equal those of the exact definition.
+    rng = np.random.default_rng(17)
+    N = 64
+    offs = np.array([0.0, 2.0 ** -20, -2.0 ** -20, 2.0 ** -15, -2.0 ** -15, 2.0 ** -14, -2.0 ** -14,
+                     2.0 ** -13, -2.0 ** -13, 1.5 * 2.0 ** -13, -1.5 * 2.0 ** -13, 2.0 ** -12, -2.0 ** -12,
+                     1e-6, -1e-6, 3e-5, -3e-5])
+    ks = np.arange(-127, 127)
+    vals = (ks[:, None] + 0.5 + offs[None, :]).ravel()
+    K = vals.size + 1
+    W = np.empty((K, N), dtype=np.float32)
+    s0 = np.float16(rng.uniform(1e-3, 8e-3, N)).astype(np.float32)
+    for n in range(N):
+        col = (rng.permutation(vals) * np.float64(s0[n])).astype(np.float32)
+        W[0, n] = np.float32(127.0) * s0[n]
+        W[1:, n] = np.clip(col, -W[0, n], W[0, n])
+    _check(W)
+    _check(W.astype(np.float16))
