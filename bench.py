@@ -343,7 +343,8 @@ def run_native(args, ws, rank, local):
             "roofline": {"bound": "tensor", "achieved": round(pf_tflops, 1), "peak": tf_sustained,
                          "unit": "TFLOP/s", "frac": round(pf_tflops / tf_sustained, 4),
                          "frac_of_burst": round(pf_tflops / tf_peak, 4),
-                         "traffic": measured_traffic("prefill_kernel", ["prefill.cuh", "common.cuh"]),
+                         "traffic": measured_traffic("prefill2_kernel", ["prefill2.cuh", "common.cuh"]),
+                         "kernel": "w8::prefill2::prefill2_kernel (CTA pairs)",
                          "peak_source": f"{peak_src} bf16_tflops_sustained (cuBLAS loop under the power cap) "
                                         f"x fp16/bf16 nominal ratio 1; burst {tf_peak}"},
         },

@@ -124,9 +124,9 @@ int w8_unpack(const uint8_t *packed, int64_t K, int64_t N, int8_t *q, void *stre
 /*
  * w8a16_workspace_bytes -- device scratch w8a16_linear needs for this shape
  * on the CURRENT device (it depends on the SM count).  0 means none.  The
- * decode path (M <= 16) splits the reduction over K across thread blocks
- * and needs room for fp32 partial sums plus one int32 counter per 128
- * output channels.
+ * weight-streaming path (M <= 64) splits the reduction over K across
+ * thread blocks and needs room for fp32 partial sums (a fixed 64 KB per
+ * multiprocessor) plus one int32 counter per 128 output channels.
  */
 size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
 
@@ -139,10 +139,10 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *   bias       [N] fp16 or NULL.
  *   Y          [M, N] fp16 output; must not overlap X, packed or scales.
  *   M >= 0 (0 is a no-op; X and Y may then be NULL); K >= 1 with
- *   K % 8 == 0; N >= 1 with N % 8 == 0.  For M <= 16 the number of 8 KB
+ *   K % 8 == 0; N >= 1 with N % 8 == 0.  For M <= 64 the number of 8 KB
  *   weight tiles times (multiprocessors + 1) must stay below 2^32 (weights
  *   up to about 230 GB on a B200), else W8_ERR_SHAPE.
- * Stream ordering: for M <= 16 the kernel is launched with programmatic
+ * Stream ordering: for M <= 64 the kernel is launched with programmatic
  *   stream serialization, so its prologue and an L2 prefetch of its first
  *   weight tiles may overlap the previous kernel in the stream; it reads X
  *   and writes Y, the workspace and the counters only after that kernel has
@@ -154,9 +154,11 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *              Calls sharing one workspace must not run concurrently on
  *              the device.  After a call whose device wait ran out (see
  *              w8_device_status) the workspace must be zeroed again.
- * Kernel choice (internal): M <= 16 streams the weight once with a
- * split-K decode kernel (HBM-bound); larger M runs a tcgen05 tensor-core
- * kernel with the widened weight tile held in tensor memory.
+ * Kernel choice (internal): M <= 64 streams the weight once with a
+ * split-K kernel on the legacy tensor-core path (HBM-bound up to about 32
+ * tokens); larger M runs a tcgen05 tensor-core kernel on pairs of SMs
+ * (clusters of two thread blocks) with the widened weight tile held in
+ * tensor memory.
  * Accuracy: |Y - Y_exact| <= 2^-9 |Y_exact| + 1e-3 rms(Y_exact).
  * Errors: W8_ERR_NULL, W8_ERR_SHAPE, W8_ERR_ALIGN, W8_ERR_WORKSPACE,
  *         W8_ERR_ALIAS, W8_ERR_DEVICE, W8_ERR_CUDA.

@@ -36,6 +36,15 @@ enum WaitSite : unsigned {
     SITE_PF_DFULL = 0x36,
     SITE_PF_DRAIN = 0x37,
     SITE_PF_XEMPTY = 0x38,
+    SITE_P2_WEMPTY = 0x40,
+    SITE_P2_XEMPTY = 0x41,
+    SITE_P2_WFULL = 0x42,
+    SITE_P2_XFULL = 0x43,
+    SITE_P2_AEMPTY = 0x44,
+    SITE_P2_AFULL = 0x45,
+    SITE_P2_DEMPTY = 0x46,
+    SITE_P2_DFULL = 0x47,
+    SITE_P2_DRAIN = 0x48,
     SITE_SELFTEST = 0xEE,
 };
 
@@ -276,6 +285,14 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
 }
+// Arrive once on an mbarrier of some CTA of the cluster with the default
+// (CTA-scope) semantics.  For signals whose data is ordered by other means
+// -- tensor-memory stores and loads completed with tcgen05.wait and fenced
+// with tcgen05.fence::before_thread_sync -- this avoids the cost of a
+// cluster-scope release (about a microsecond per arrive).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar_addr, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -313,6 +330,58 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
+}
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// 2-D tensor load into this CTA's shared memory whose completion is
+// counted on `bar_cluster`, an mbarrier of either CTA of the pair
+// (shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void *dst_smem, const CUtensorMap *map, int32_t x,
+                                                 int32_t y, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+// D[tmem, both CTAs] (+)= A[tmem, both CTAs] * B[smem desc, both CTAs]:
+// M = 256 (128 rows in each CTA), issued by one thread of the pair's
+// first CTA.
+__device__ __forceinline__ void tc_mma_ts_f16_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                   uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive once on the mbarrier at `bar`'s offset in each CTA of `cta_mask`
+// when all prior pair MMAs of this thread have completed.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
 }
 
 // ---------------------------------------------------------------- named barriers

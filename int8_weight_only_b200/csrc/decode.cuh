@@ -1,4 +1,4 @@
-// Decode-regime W8A16 linear (M <= 16 tokens): Y = X . dequant(q) (+ bias).
+// Decode-regime W8A16 linear (M <= 64 tokens): Y = X . dequant(q) (+ bias).
 //
 // For few tokens the cost is streaming the int8 weight from HBM once
 // (TPU-MLIR ChatGLM2 W8A16 article, section 4: when the left matrix is
@@ -14,9 +14,10 @@
 //    warps each own 16 of the tile's 128 channels.
 //  - Consumers widen int8 to fp16 in registers (prmt into the exponent
 //    pattern of 1024, then one fp16x2 subtraction) and accumulate in fp32
-//    with mma.sync m16n8k16 (channels as the MMA rows, tokens as its 8 or
-//    16 columns), so conversion plus multiply-add stay a small fraction of
-//    the issue budget even at 16 tokens.  The stage's tiles are unrolled and
+//    with mma.sync m16n8k16 (channels as the MMA rows, tokens as its 8
+//    columns, up to 8 token tiles), so conversion plus multiply-add stay a
+//    small fraction of the issue budget; up to 64 tokens the weight stream
+//    still sets the pace.  The stage's tiles are unrolled and
 //    each 16-wide k slice has its own accumulator, so the mma results do not
 //    form one long dependency chain.
 //  - Only a CTA's first and last channel block can be split with other
@@ -39,22 +40,33 @@ namespace decode {
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kTilesPerStage = 4;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;
 constexpr int kTileBytes = 8192;
 constexpr int kStageW = kTilesPerStage * kTileBytes;
+constexpr int kMaxTokens = 64;     // MT <= 8 token tiles of 8
 
+// MT = token tiles of 8 (1, 2, 4 or 8: up to 8, 16, 32 or 64 tokens).
 template <int MT>
 struct Cfg {
     static constexpr int kXRows = 8 * MT;                // token rows per X box
     static constexpr int kXBoxBytes = kXRows * 128;      // box {64 fp16, kXRows}
     static constexpr int kStageX = kTilesPerStage * kXBoxBytes;
     static constexpr int kStageBytes = kStageW + kStageX;
+    static constexpr int kStages = MT <= 4 ? 4 : 3;      // ring within shared memory
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
     static constexpr int kPartialFloats = kConsumerWarps * 4 * MT * 32;   // per slot
+    // independent accumulators per token tile: one per 16-wide k slice for
+    // few tokens (otherwise one long mma chain), one when the token tiles
+    // already give enough independent chains
+    static constexpr int kNS = MT <= 2 ? 4 : 1;
 };
 
-// Workspace: [partials: 2 slots per SM][counters: one int32 per channel block]
-constexpr int kMaxPartialFloats = Cfg<2>::kPartialFloats;
+// Workspace: [partials: 2 slots per SM, sized for MT = 8][counters: one
+// int32 per channel block].  The same size for every M and N, so the
+// counters always sit at the same offset.
+constexpr int kMaxPartialFloats = Cfg<8>::kPartialFloats;
+// Partial slot size when at most 16 tokens are allowed.
+constexpr int kPartialFloats16 = Cfg<2>::kPartialFloats;
 
 struct Params {
     const uint8_t *packed;
@@ -117,14 +129,18 @@ __device__ __forceinline__ void store_y(const Params &p, uint32_t b, int warp, i
     }
 }
 
-// Sum the four per-k-slice accumulators of each token tile.
-template <int MT>
-__device__ __forceinline__ void fold(const float (&acc)[MT][4][4], float (&out)[MT][4]) {
+// Sum the per-k-slice accumulators of each token tile.
+template <int MT, int NS>
+__device__ __forceinline__ void fold(const float (&acc)[MT][NS][4], float (&out)[MT][4]) {
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            out[mt][e] = (acc[mt][0][e] + acc[mt][1][e]) + (acc[mt][2][e] + acc[mt][3][e]);
+        for (int e = 0; e < 4; ++e) {
+            if constexpr (NS == 4)
+                out[mt][e] = (acc[mt][0][e] + acc[mt][1][e]) + (acc[mt][2][e] + acc[mt][3][e]);
+            else
+                out[mt][e] = acc[mt][0][e];
+        }
 }
 
 template <int MT>
@@ -134,7 +150,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t full[kStages], empty[kStages];
+    __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
     __shared__ uint64_t fix_bar;
     __shared__ int last_flag[2];   // [0]: partner part ready; [1]: last contributor
 
@@ -146,7 +162,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     const uint32_t t_end = range_start(cta + 1, p.T, p.G);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
@@ -165,7 +181,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             // The weights are not written by the previous kernel in any
             // sane use, but only an L2 prefetch (never stale) runs before
             // the wait: the first ring's worth of this CTA's range.
-            const uint32_t pre_tiles = min(t_end - t_begin, (uint32_t)(kStages * kTilesPerStage));
+            const uint32_t pre_tiles = min(t_end - t_begin, (uint32_t)(C::kStages * kTilesPerStage));
             prefetch_l2(p.packed + (size_t)t_begin * kTileBytes, pre_tiles * kTileBytes);
             pdl_wait();
             const uint64_t policy = policy_evict_first();
@@ -186,12 +202,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                 kb += cnt;
                 if (kb == KB) kb = 0;
                 ++issued;
-                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
             // every copy this CTA issued has landed before the CTA can exit
             // (normally long since consumed; matters only after a timeout)
-            for (int i = 0; i < kStages && i < issued; ++i) {
-                if (--stage < 0) { stage = kStages - 1; phase ^= 1u; }
+            for (int i = 0; i < C::kStages && i < issued; ++i) {
+                if (--stage < 0) { stage = C::kStages - 1; phase ^= 1u; }
                 mbar_wait(&full[stage], phase, SITE_DEC_DRAIN, 10000000ull);
             }
         }
@@ -213,13 +229,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         x_off[mt][1] = m * 128 + (((2 * tq + 1) ^ (m & 7)) << 4);
     }
 
-    // one accumulator per 16-wide k slice of the tile: four independent
-    // mma chains instead of one
-    float acc[MT][4][4];
+    // independent accumulators (see Cfg::kNS)
+    constexpr int NS = C::kNS;
+    float acc[MT][NS][4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
+        for (int jj = 0; jj < NS; ++jj)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[mt][jj][e] = 0.0f;
 
@@ -300,7 +316,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                         const uint4 &xq = xv[mt][jj >> 1];
                         const uint32_t b0 = (jj & 1) ? xq.z : xq.x;
                         const uint32_t b1 = (jj & 1) ? xq.w : xq.y;
-                        mma_16816(acc[mt][jj], a0, a1, a2, a3, b0, b1);
+                        mma_16816(acc[mt][jj % NS], a0, a1, a2, a3, b0, b1);
                     }
                 }
             }
@@ -309,14 +325,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         if (lane == 0) mbar_arrive(&empty[stage]);
         t += cnt;
         kb += cnt;
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         if (t != t_end && kb != KB) continue;
 
         // ------------------------------------------------ end of a segment
         // This CTA's part of channel block b is done.  It is the whole block
         // if it started at K block 0 and reached the end.
         float sum[MT][4];
-        fold<MT>(acc, sum);
+        fold<MT, NS>(acc, sum);
         if (seg_whole && kb == KB) {
             store_y<MT>(p, b, warp, lane, sum);
         } else if (have_pre && b == last_b) {
@@ -375,7 +391,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
+            for (int jj = 0; jj < NS; ++jj)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[mt][jj][e] = 0.0f;
         if (kb == KB) { kb = 0; ++b; }

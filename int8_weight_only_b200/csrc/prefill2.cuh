@@ -1,0 +1,349 @@
+// Prefill-regime W8A16 linear on CTA pairs (tcgen05 cta_group::2):
+// Y = X . dequant(q) (+ bias).  The TPU-MLIR article (section 4) gives the
+// W8A16 MatMul as load -> cast int8 to F16 -> scale -> matmul -> store,
+// with the load overlapped with compute through ping-pong local memory; on
+// sm_100a the same five steps become a warp-specialised, persistent
+// pipeline in which each MMA spans the two SMs of a cluster of two CTAs.
+//
+// One thread issues a tcgen05.mma only about every 100 cycles, so the MMA
+// shape must carry enough work: 128 x 256 x 16 per SM (136 cycles) keeps
+// the tensor pipe busy where 128 x 128 x 16 (64 cycles) cannot.  A pair
+// tile is 256 channels x 256 tokens: each CTA holds its
+// own 128 channels (widened weights in its tensor memory, accumulator rows
+// in its tensor memory) and HALF of the tokens' X tile (128 x 64, 16 KB) in
+// its shared memory; one 256 x 256 x 16 MMA issued by the pair's first CTA
+// reads the A halves from both tensor memories and the B halves from both
+// shared memories.  Compared with one SM per 128 x 256 tile this halves the
+// X tile each SM pulls from L2 per K step; no TMA multicast is used.
+//
+// Roles in each CTA (16 warps):
+//   warp 0      weight producer: bulk copy of this CTA's four 8 KB packed
+//               tiles per 256-wide K step into a local 3-stage ring.
+//   warp 3      activation producer: four 2-D TMA loads of this CTA's 128
+//               tokens x 64 X halves per K step into a local 2-stage ring of
+//               64 KB slots; the completion is counted on the FIRST CTA's
+//               barrier (both CTAs' halves must land before the pair MMAs).
+//   warps 4-7   converters: widen the int8 codes into this CTA's tensor
+//               memory A buffer, then arrive on the first CTA's barrier.
+//   warp 1      (first CTA only) MMA issuer; its commits arrive on the
+//               barriers of both CTAs.
+//   warps 8-15  epilogue: drain this CTA's 128 accumulator lanes, release
+//               the accumulator on the first CTA's barrier, scale, store.
+//   warp 2      tensor-memory allocation for the pair.
+#pragma once
+
+#include "common.cuh"
+
+namespace w8 {
+namespace prefill2 {
+
+constexpr int kBNc = 128;                // channels per CTA
+constexpr int kBNp = 2 * kBNc;           // channels per pair tile (MMA M)
+constexpr int kBT = 256;                 // tokens per pair tile (MMA N)
+constexpr int kBTc = kBT / 2;            // tokens held by each CTA
+// One pipeline stage covers a 256-wide K step: four packed tiles, four
+// 64-wide X boxes and sixteen MMAs.  Every stage costs a handful of barrier
+// handoffs (a few hundred cycles each, measured: arrive, wake-up, commit),
+// so the step is made long enough (about 2200 cycles of tensor work) to
+// hide them; 64- and 128-wide steps left the tensor pipe half and a fifth
+// idle.
+constexpr int kKStep = 4;                // 64-wide K blocks per stage
+constexpr int kWStages = 3;
+constexpr int kXStages = 2;
+constexpr int kWTile = 8192;             // packed int8 tile, 128 x 64
+constexpr int kWBytes = kKStep * kWTile;
+constexpr int kXBox = kBTc * 128;        // 128 tokens x 64 fp16
+constexpr int kXBytes = kKStep * kXBox;
+constexpr int kSmemBytes = kXStages * kXBytes + kWStages * kWBytes + 1024;
+constexpr int kABuf = 2;                 // A buffers of 32 kKStep columns
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAcol0 = kBT;         // first A buffer column
+constexpr int kThreads = 512;
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kIdesc = idesc_f16_f32(kBNp, kBT);
+constexpr uint16_t kBoth = 0x3;          // CTA mask of the pair
+
+static_assert(kXBox % 1024 == 0 && kWBytes % 1024 == 0, "stage alignment");
+static_assert(kAcol0 + 32 * kKStep * kABuf <= kTmemCols, "tensor memory budget");
+static_assert(kSmemBytes <= 227 * 1024 - 512, "shared memory budget");
+
+struct Params {
+    const uint8_t *packed;
+    const uint16_t *scales;
+    const uint16_t *bias;   // may be null
+    uint16_t *Y;
+    int M;
+    int64_t N;
+    int NB;        // ceil(N/128): packed channel blocks
+    int KB;        // ceil(K/64)
+    int KS;        // ceil(KB/4): 256-wide K steps
+    int TT;        // token tiles = ceil(M/256)
+    int64_t tiles; // ceil(NB/2) * TT pair tiles
+};
+
+struct Ring {
+    int s = 0;
+    uint32_t ph = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++s == n) { s = 0; ph ^= 1u; }
+    }
+    __device__ __forceinline__ void prev(int n) {
+        if (--s < 0) { s = n - 1; ph ^= 1u; }
+    }
+};
+
+// grid = 2 x pairs CTAs, cluster dims (2, 1, 1), kThreads threads,
+// kSmemBytes dynamic shared memory.  tmap_x: X [M, K] fp16, box {64, 128},
+// 128-byte swizzle.
+__global__ void __launch_bounds__(kThreads, 1)
+prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *x_ring = base;                                  // kXStages x 16 KB
+    uint8_t *w_ring = base + kXStages * kXBytes;             // kWStages x 8 KB
+    __shared__ uint64_t w_full[kWStages], w_empty[kWStages];
+    __shared__ uint64_t x_full[kXStages], x_empty[kXStages];
+    __shared__ uint64_t a_full[kABuf], a_empty[kABuf];
+    __shared__ uint64_t d_full, d_empty, drain;
+    __shared__ uint32_t tmem_base_sh;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();     // 0: issues the pair MMAs
+    const int64_t pair0 = blockIdx.x >> 1;
+    const int64_t pstep = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kWStages; ++i) {
+            mbar_init(&w_full[i], 1);
+            mbar_init(&w_empty[i], 4);         // this CTA's converter warps
+        }
+        for (int i = 0; i < kXStages; ++i) {
+            mbar_init(&x_full[i], 1);          // first CTA: expect both halves
+            mbar_init(&x_empty[i], 1);         // pair MMA commit
+        }
+        for (int i = 0; i < kABuf; ++i) {
+            mbar_init(&a_full[i], 8);          // converter warps of both CTAs
+            mbar_init(&a_empty[i], 1);
+        }
+        mbar_init(&d_full, 1);
+        mbar_init(&d_empty, 2 * kEpiWarps);    // epilogue warps of both CTAs
+        mbar_init(&drain, 1);
+        fence_barrier_init();
+        prefetch_tensormap(&tmap_x);
+    }
+    if (warp == 2) {
+        tmem_alloc_pair(&tmem_base_sh, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();   // barriers initialised in both CTAs, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    // the first CTA's copy of a barrier, as a shared::cluster address
+    auto leader = [](uint64_t *bar) -> uint32_t { return mapa_shared(smem_u32(bar), 0); };
+
+    if (warp == 0) {
+        // ---------------------------------------------------- weight producer
+        if (lane == 0) {
+            Ring r;
+            int issued = 0;
+            bool ok = true;
+            for (int64_t pt = pair0; pt < p.tiles && ok; pt += pstep) {
+                const int64_t blk = (pt / p.TT) * 2 + rank;
+                const bool valid = blk < p.NB;
+                const uint8_t *wsrc = p.packed + blk * p.KB * (int64_t)kWTile;
+                for (int ks = 0; ks < p.KS; ++ks) {
+                    const int cnt = min(kKStep, p.KB - kKStep * ks);   // tiles in this step
+                    if (!mbar_wait(&w_empty[r.s], r.ph ^ 1u, SITE_P2_WEMPTY)) { ok = false; break; }
+                    if (valid) {
+                        mbar_arrive_expect_tx(&w_full[r.s], cnt * kWTile);
+                        bulk_g2s(w_ring + r.s * kWBytes, wsrc + (int64_t)kKStep * ks * kWTile, cnt * kWTile,
+                                 &w_full[r.s]);
+                        ++issued;
+                    } else {
+                        mbar_arrive(&w_full[r.s]);   // no block: converters write zeros
+                    }
+                    r.next(kWStages);
+                }
+            }
+            for (int i = 0; i < kWStages && i < issued; ++i) {
+                r.prev(kWStages);
+                mbar_wait(&w_full[r.s], r.ph, SITE_P2_DRAIN, 10000000ull);
+            }
+        }
+    } else if (warp == 3) {
+        // ---------------------------------------------------- activation producer
+        if (lane == 0) {
+            Ring r;
+            int issued = 0;
+            bool ok = true;
+            for (int64_t pt = pair0; pt < p.tiles && ok; pt += pstep) {
+                const int tb = (int)(pt % p.TT);
+                for (int ks = 0; ks < p.KS; ++ks) {
+                    const int cnt = min(kKStep, p.KB - kKStep * ks);
+                    if (!mbar_wait(&x_empty[r.s], r.ph ^ 1u, SITE_P2_XEMPTY)) { ok = false; break; }
+                    if (rank == 0) mbar_arrive_expect_tx(&x_full[r.s], 2 * cnt * kXBox);
+                    for (int t = 0; t < cnt; ++t)
+                        tma_load_2d_pair(x_ring + r.s * kXBytes + t * kXBox, &tmap_x, (kKStep * ks + t) * 64,
+                                         tb * kBT + (int)rank * kBTc, leader(&x_full[r.s]));
+                    ++issued;
+                    r.next(kXStages);
+                }
+            }
+            // every X half has landed before the pair can leave: the first
+            // CTA sees both halves complete on its barrier; the MMA issuer
+            // consumed them, or after a timeout the final cluster barrier
+            // below orders the exit after this wait in the first CTA
+            if (rank == 0) {
+                for (int i = 0; i < kXStages && i < issued; ++i) {
+                    r.prev(kXStages);
+                    mbar_wait(&x_full[r.s], r.ph, SITE_P2_DRAIN, 10000000ull);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer (first CTA)
+        if (lane == 0 && rank == 0) {
+            Ring xr, ar;
+            int it = 0;
+            bool ok = true;
+            for (int64_t pt = pair0; pt < p.tiles && ok; pt += pstep, ++it) {
+                if (!mbar_wait(&d_empty, (it & 1) ^ 1u, SITE_P2_DEMPTY)) { ok = false; break; }
+                tc_fence_after();
+                for (int ks = 0; ks < p.KS; ++ks) {
+                    const int cnt = min(kKStep, p.KB - kKStep * ks);
+                    if (!mbar_wait(&x_full[xr.s], xr.ph, SITE_P2_XFULL)) { ok = false; break; }
+                    if (!mbar_wait(&a_full[ar.s], ar.ph, SITE_P2_AFULL)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_tmem = tmem + kAcol0 + 32 * kKStep * ar.s;
+                    const uint32_t x_addr = smem_u32(x_ring + xr.s * kXBytes);
+                    for (int t = 0; t < cnt; ++t) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            tc_mma_ts_f16_pair(tmem, a_tmem + 32 * t + 8 * j,
+                                               smem_desc_kmajor_sw128(x_addr + t * kXBox + 32 * j), kIdesc,
+                                               (ks | t | j) != 0);
+                    }
+                    tc_commit_pair_mc(&x_empty[xr.s], kBoth);
+                    tc_commit_pair_mc(&a_empty[ar.s], kBoth);
+                    xr.next(kXStages);
+                    ar.next(kABuf);
+                }
+                if (!ok) break;
+                tc_commit_pair_mc(&d_full, kBoth);
+            }
+            // every pair MMA is complete before either CTA frees its TMEM
+            tc_commit_pair(&drain);
+            mbar_wait(&drain, 0, SITE_P2_DRAIN);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ---------------------------------------------------- converters
+        const int q4 = warp & 3;
+        const int r = 32 * q4 + lane;         // channel within this CTA's block
+        const int h = (r >> 1) & 3;
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
+        Ring wr, ar;
+        bool ok = true;
+        for (int64_t pt = pair0; pt < p.tiles && ok; pt += pstep) {
+            const bool valid = (pt / p.TT) * 2 + rank < p.NB;
+            for (int ks = 0; ks < p.KS; ++ks) {
+                const int cnt = min(kKStep, p.KB - kKStep * ks);
+                if (!warp_all(mbar_wait(&w_full[wr.s], wr.ph, SITE_P2_WFULL))) { ok = false; break; }
+                uint4 c[kKStep][4];
+#pragma unroll
+                for (int t = 0; t < kKStep; ++t) {
+                    if (valid && t < cnt) {
+                        const uint8_t *row = w_ring + wr.s * kWBytes + t * kWTile + r * 64;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) c[t][i] = *reinterpret_cast<const uint4 *>(row + ((i ^ h) << 4));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            c[t][i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&w_empty[wr.s]);
+                if (!warp_all(mbar_wait(&a_empty[ar.s], ar.ph ^ 1u, SITE_P2_AEMPTY))) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int t = 0; t < kKStep; ++t) {
+                    uint32_t v[32];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t w[4] = {c[t][i].x, c[t][i].y, c[t][i].z, c[t][i].w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            v[8 * i + 2 * j] = unbias2(widen_lo2(w[j]));
+                            v[8 * i + 2 * j + 1] = unbias2(widen_hi2(w[j]));
+                        }
+                    }
+                    tmem_st_32x32b_x32(lane_addr + kAcol0 + 32 * kKStep * ar.s + 32 * t, v);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(leader(&a_full[ar.s]));
+                wr.next(kWStages);
+                ar.next(kABuf);
+            }
+        }
+    } else if (warp >= 8) {
+        // ---------------------------------------------------- epilogue
+        const int q4 = warp & 3;
+        const int half = (warp - 8) >> 2;     // token columns [128 half, 128 half + 128)
+        const int r = 32 * q4 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16) + 128 * half;
+        int it = 0;
+        for (int64_t pt = pair0; pt < p.tiles; pt += pstep, ++it) {
+            if (!warp_all(mbar_wait(&d_full, it & 1, SITE_P2_DFULL))) break;
+            tc_fence_after();
+            const int64_t blk = (pt / p.TT) * 2 + rank;
+            const int tb = (int)(pt % p.TT);
+            const int64_t n = blk * kBNc + r;
+            const bool n_ok = n < p.N;
+            const float sc = n_ok ? __half2float(__ushort_as_half(p.scales[n])) : 0.0f;
+            const float bi = (n_ok && p.bias) ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
+            uint32_t y2[64];
+#pragma unroll
+            for (int cchunk = 0; cchunk < 4; ++cchunk) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(lane_addr + 32 * cchunk, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const __half2 hv = __floats2half2_rn(fmaf(__uint_as_float(v[2 * i]), sc, bi),
+                                                         fmaf(__uint_as_float(v[2 * i + 1]), sc, bi));
+                    y2[16 * cchunk + i] = *reinterpret_cast<const uint32_t *>(&hv);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(leader(&d_empty));
+            if (n_ok) {
+                const int m0 = tb * kBT + 128 * half;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const int m = m0 + 2 * i;
+                    if (m < p.M) p.Y[(int64_t)m * p.N + n] = (uint16_t)(y2[i] & 0xFFFFu);
+                    if (m + 1 < p.M) p.Y[(int64_t)(m + 1) * p.N + n] = (uint16_t)(y2[i] >> 16);
+                }
+            }
+        }
+    }
+
+    // neither CTA frees the pair's tensor memory, nor leaves while the
+    // other may still signal its barriers, before both are done
+    tc_fence_before();
+    cluster_sync_all();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+}  // namespace prefill2
+}  // namespace w8

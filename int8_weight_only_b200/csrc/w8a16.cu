@@ -1,6 +1,6 @@
 // libw8a16.so: the C ABI declared in include/w8a16.h.  Host code only
 // validates arguments, builds TMA tensor maps and launches the kernels in
-// quantize.cuh, prepack.cuh, decode.cuh and prefill.cuh on the caller's
+// quantize.cuh, prepack.cuh, decode.cuh and prefill2.cuh on the caller's
 // stream.  Nothing here allocates device memory or synchronizes (except the
 // w8_device_status diagnostic).
 #include <cudaTypedefs.h>
@@ -12,7 +12,7 @@
 #include "../../include/w8a16.h"
 #include "common.cuh"
 #include "decode.cuh"
-#include "prefill.cuh"
+#include "prefill2.cuh"
 #include "prepack.cuh"
 #include "quantize.cuh"
 
@@ -26,6 +26,7 @@ struct DeviceInfo {
     bool ready = false;
     int status = W8_OK;   // W8_ERR_DEVICE if not sm_100
     int sms = 0;
+    int pairs = 0;   // resident prefill CTA pairs (0 = not yet queried)
     // resident quantize clusters per cluster size (0 = not yet queried)
     int qclusters_f32[quant::kMaxCluster + 1] = {};
     int qclusters_f16[quant::kMaxCluster + 1] = {};
@@ -57,9 +58,17 @@ int device_info(DeviceInfo **out) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          decode::Cfg<2>::kSmemBytes);
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(prefill::prefill_kernel,
+                e = cudaFuncSetAttribute(decode::decode_kernel<4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         prefill::kSmemBytes);
+                                         decode::Cfg<4>::kSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(decode::decode_kernel<8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         decode::Cfg<8>::kSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(prefill2::prefill2_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         prefill2::kSmemBytes);
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(quant::quantize_kernel<float>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, quant::kSmemBytes);
@@ -183,6 +192,80 @@ int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_
     return launch_status();
 }
 
+// Programmatic dependent launch: this kernel's prologue and an L2 prefetch
+// of its first weight tiles overlap the previous kernel in the stream.
+template <int MT>
+int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.G, 1, 1);
+    cfg.blockDim = dim3(decode::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = decode::Cfg<MT>::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode::decode_kernel<MT>, map, p) != cudaSuccess) {
+        cudaGetLastError();
+        return W8_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+// Tensor-core linear for M > 64 on CTA pairs (prefill2.cuh).
+int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
+                    const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N, cudaStream_t st) {
+    CUtensorMap map;
+    int rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
+                         prefill2::kBTc, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != W8_OK) return rc;
+    prefill2::Params p;
+    p.packed = packed;
+    p.scales = scales;
+    p.bias = bias;
+    p.Y = Y;
+    p.M = (int)M;
+    p.N = N;
+    p.NB = (int)cdiv(N, 128);
+    p.KB = (int)cdiv(K, 64);
+    p.KS = (int)cdiv(p.KB, prefill2::kKStep);
+    p.TT = (int)cdiv(M, prefill2::kBT);
+    p.tiles = cdiv(p.NB, 2) * p.TT;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(prefill2::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = prefill2::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int resident = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (d->pairs == 0) {
+            cfg.gridDim = dim3((unsigned)d->sms, 1, 1);
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, prefill2::prefill2_kernel, &cfg) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                n = d->sms / 2;
+            }
+            d->pairs = n;
+        }
+        resident = d->pairs;
+    }
+    const int64_t pairs = std::min<int64_t>(p.tiles, resident);
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel, map, p) != cudaSuccess) {
+        cudaGetLastError();
+        return W8_ERR_CUDA;
+    }
+    return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -288,7 +371,7 @@ static size_t decode_workspace(int sms, int64_t K, int64_t N) {
 }
 
 size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N) {
-    if (M < 1 || M > 16 || K < 1 || N < 1) return 0;
+    if (M < 1 || M > decode::kMaxTokens || K < 1 || N < 1) return 0;
     DeviceInfo *d = nullptr;
     if (device_info(&d) != W8_OK) return 0;
     return decode_workspace(d->sms, K, N);
@@ -318,12 +401,12 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
     const int KB = (int)cdiv(K, 64);
     const int64_t NB = cdiv(N, 128);
 
-    if (M <= 16) {
+    if (M <= decode::kMaxTokens) {
         const size_t need = decode_workspace(d->sms, K, N);
         if (!workspace || workspace_bytes < need) return W8_ERR_WORKSPACE;
         if (overlap(workspace, need, Y, ybytes) || overlap(workspace, need, X, (size_t)M * K * 2))
             return W8_ERR_ALIAS;
-        const int MT = M <= 8 ? 1 : 2;
+        const int MT = M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8;
         CUtensorMap map;
         rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
                          8 * MT, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -344,44 +427,15 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
         if ((uint64_t)T * (uint64_t)(G + 1) >= (1ull << 32)) return W8_ERR_SHAPE;
         p.T = (uint32_t)T;
         p.G = (uint32_t)G;
-        // programmatic dependent launch: this kernel's prologue and an L2
-        // prefetch of its first weight tiles overlap the previous kernel
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)G, 1, 1);
-        cfg.blockDim = dim3(decode::kThreads, 1, 1);
-        cfg.dynamicSmemBytes = MT == 1 ? decode::Cfg<1>::kSmemBytes : decode::Cfg<2>::kSmemBytes;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const cudaError_t e = MT == 1 ? cudaLaunchKernelEx(&cfg, decode::decode_kernel<1>, map, p)
-                                      : cudaLaunchKernelEx(&cfg, decode::decode_kernel<2>, map, p);
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            return W8_ERR_CUDA;
+        switch (MT) {
+            case 1: return launch_decode<1>(map, p, st);
+            case 2: return launch_decode<2>(map, p, st);
+            case 4: return launch_decode<4>(map, p, st);
+            default: return launch_decode<8>(map, p, st);
         }
-        return launch_status();
     }
 
-    CUtensorMap map;
-    rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
-                     prefill::kBT, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (rc != W8_OK) return rc;
-    prefill::Params p;
-    p.packed = packed;
-    p.scales = scales;
-    p.bias = bias;
-    p.Y = Y;
-    p.M = (int)M;
-    p.N = N;
-    p.KB = KB;
-    p.TT = (int)cdiv(M, prefill::kBT);
-    p.tiles = NB * p.TT;
-    const int grid = (int)std::min<int64_t>(p.tiles, d->sms);
-    prefill::prefill_kernel<<<grid, prefill::kThreads, prefill::kSmemBytes, st>>>(map, p);
-    return launch_status();
+    return launch_prefill2(d, X, packed, scales, bias, Y, M, K, N, st);
 }
 
 // ---------------------------------------------------------------- diagnostics
@@ -427,7 +481,7 @@ int w8_device_status(void *stream, uint32_t *out) {
 // one per 128-channel block, up to W8_STATIC_MAX_N / 128].
 namespace {
 constexpr size_t kStaticPartialBytes =
-    (size_t)2 * W8_STATIC_MAX_SMS * decode::kMaxPartialFloats * sizeof(float);
+    (size_t)2 * W8_STATIC_MAX_SMS * decode::kPartialFloats16 * sizeof(float);
 constexpr size_t kStaticCounterBytes = (size_t)(W8_STATIC_MAX_N / 128) * sizeof(int);
 static_assert(kStaticPartialBytes + kStaticCounterBytes == (size_t)W8_STATIC_SCRATCH_BYTES,
               "header size of the static scratch");

@@ -31,21 +31,21 @@ def _check_full(M, K, N, tid, bias=True):
     return assert_close(Yg, Yref, f"M={M} K={K} N={N}")
 
 
-# ---------------------------------------------------------------- decode (M <= 16)
+# ---------------------------------------------------------------- weight streaming (M <= 64)
 DECODE_SHAPES = [(256, 512), (64, 8), (200, 136), (1024, 1032), (4096, 4608), (13696, 264)]
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16, 17, 31, 32, 33, 48, 64])
 @pytest.mark.parametrize("K,N", DECODE_SHAPES)
 def test_decode_matches_oracle(M, K, N):
     _check_full(M, K, N, 2000 + K + N + M, bias=(M % 2 == 1))
 
 
-# ---------------------------------------------------------------- prefill (M > 16)
+# ---------------------------------------------------------------- tensor cores (M > 64)
 PREFILL_SHAPES = [(256, 512), (64, 136), (520, 264), (4096, 384)]
 
 
-@pytest.mark.parametrize("M", [17, 64, 128, 129, 300])
+@pytest.mark.parametrize("M", [65, 128, 129, 256, 257, 300])
 @pytest.mark.parametrize("K,N", PREFILL_SHAPES)
 def test_prefill_matches_oracle(M, K, N):
     _check_full(M, K, N, 3000 + K + N + M, bias=(M % 2 == 0))
@@ -109,8 +109,9 @@ def test_deterministic_across_calls():
 
 def test_workspace_reused_across_shapes():
     # the split-K counters are reset by each call, so one workspace serves
-    # calls of different shapes back to back
-    for (M, K, N) in [(1, 4096, 512), (3, 64, 8), (16, 1000, 1032), (1, 4096, 512)]:
+    # calls of different shapes and token counts back to back
+    for (M, K, N) in [(1, 4096, 512), (3, 64, 8), (16, 1000, 1032), (64, 2048, 4104), (1, 4096, 512),
+                      (40, 4096, 27392), (9, 13696, 264)]:
         _check_full(M, K, N, 3700 + K + N)
 
 
@@ -126,7 +127,8 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(m.W8Error) as e:
         m.linear(to_gpu(X), packed, s, workspace=ws)
     assert e.value.status == -5
-    assert m.workspace_bytes(17, 256, 512) == 0
+    assert m.workspace_bytes(64, 256, 512) > 0
+    assert m.workspace_bytes(65, 256, 512) == 0
 
 
 def test_empty_batch():
@@ -159,7 +161,7 @@ def test_chatglm2_h_to_4h_decode_full():
     assert_close(Yg, oracle.linear(X, qall, sall), "h-to-4h decode all")
 
 
-@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16, 32, 64])
 def test_chatglm2_decode_layer_sampled(M):
     rng = np.random.default_rng(M)
     for i, (K, N) in enumerate(synthetic.WORKLOADS["chatglm2_decode_set"]["matrices"]):
