@@ -304,6 +304,58 @@ def run_native(args, ws, rank, local):
     t_e2e = timed_replays(g_e2e, n_rep, stream, ws, device, sampler)
     e2e_value = ws * weight_bytes * steps_done / t_e2e / 1e9
 
+    # ---- the ChatGLM2-6B decode layer set: 28 layers x 4 linears (QKV,
+    # dense, h-to-4h, 4h-to-h), each call on its own weight buffer (5.7 GB
+    # in all, so nothing is served from L2), chained in one CUDA graph
+    decode_set = {}
+    if not args.no_decode_set:
+        spec = synthetic.WORKLOADS["chatglm2_decode_set"]
+        mats, layers = spec["matrices"], spec["layers"]
+        packed_set, scale_set = [], []
+        for i, (Kd, Nd) in enumerate(mats):
+            Wd = torch.from_numpy(synthetic.weights(Kd, Nd, seed, synthetic.tensor_id(3, 0, i, 0),
+                                                    outlier_frac=spec["outlier_frac"])).to(device)
+            with torch.cuda.stream(stream):
+                qd, sd = w8.quantize(Wd)
+                pd = w8.prepack(qd)
+            torch.cuda.synchronize()
+            del Wd, qd
+            # distinct buffers per layer (copies of one synthetic layer)
+            packed_set.append([pd] + [pd.clone() for _ in range(layers - 1)])
+            scale_set.append(sd)
+        set_bytes = layers * sum(Kd * Nd for Kd, Nd in mats)
+        for Md in (1, 16):
+            Xs = [torch.from_numpy(synthetic.activations(Md, Kd, seed, synthetic.tensor_id(3, Md, i, 1))).to(device)
+                  for i, (Kd, Nd) in enumerate(mats)]
+            Ys = [torch.empty((Md, Nd), dtype=torch.float16, device=device) for Kd, Nd in mats]
+            wsd = torch.zeros((max(w8.workspace_bytes(Md, Kd, Nd, device) for Kd, Nd in mats),),
+                              dtype=torch.uint8, device=device)
+
+            def set_round():
+                for layer in range(layers):
+                    for i in range(len(mats)):
+                        w8.linear(Xs[i], packed_set[i][layer], scale_set[i], out=Ys[i], workspace=wsd)
+
+            with torch.cuda.stream(stream):
+                set_round()   # first calls outside capture
+            torch.cuda.synchronize()
+            g_set = capture(set_round, stream)
+            for _ in range(3):
+                with torch.cuda.stream(stream):
+                    g_set.replay()
+            torch.cuda.synchronize()
+            reps = max(10, args.set_reps)
+            t_set = timed_replays(g_set, reps, stream, ws, device, sampler) / reps
+            decode_set[f"M={Md}"] = {
+                "us_per_layer_set": round(t_set * 1e6, 1),
+                "us_per_layer": round(t_set * 1e6 / layers, 2),
+                "weight_GBps": round(set_bytes / t_set / 1e9, 1),
+                "frac_hbm": round(set_bytes / t_set / 1e9 / hbm_peak, 4),
+                "linears": layers * len(mats), "weight_bytes": set_bytes,
+            }
+            del g_set
+        del packed_set
+
     clocks = sampler.stop()
 
     out = {
@@ -360,6 +412,9 @@ def run_native(args, ws, rank, local):
                 "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()),
                 "how": "public API call per step with pinned-host X->device and Y->host copies, "
                        "graph-replayed"},
+        "decode_set": ({"workload": "ChatGLM2-6B decode linears, 28 layers x (QKV 4096x4608, dense 4096x4096, "
+                                    "h-to-4h 4096x27392, 4h-to-h 13696x4096), distinct weight buffers, one CUDA graph",
+                        **decode_set} if decode_set else None),
         "gpu_launches": steps_done,
         "clocks": clocks,
     }
@@ -470,6 +525,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-cols", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-set", action="store_true",
+                    help="skip the 28-layer decode set measurement")
+    ap.add_argument("--set-reps", type=int, default=100)
     ap.add_argument("--profile", choices=["decode", "decode16", "prefill", "quantize", "prepack"],
                     help="run --steps plain launches of one kernel (for ncu) and exit")
     args = ap.parse_args()

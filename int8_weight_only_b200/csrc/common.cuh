@@ -87,6 +87,15 @@ __device__ __forceinline__ int ld_acquire_gpu(const int *p) {
     return v;
 }
 
+// Atomic add at GPU scope with acquire-release semantics: publishes what
+// this thread (and, through a preceding CTA barrier, its CTA) wrote before
+// it, and orders what it reads after it.
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // ---------------------------------------------------------------- smem
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -359,30 +359,54 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             const uint32_t j_first = owner_of(b * KB, p.T, p.G);
             const uint32_t j_last = owner_of((b + 1) * KB - 1, p.T, p.G);
             if (threadIdx.x == 0) {
-                __threadfence();   // with the barrier above: every thread's part
-                const int old = atomicAdd(&p.counters[b], 1);
+                // release (with the barrier above: every thread's part) and
+                // acquire (the parts are read after the count) in one atomic
+                const int old = atomic_add_acq_rel_gpu(&p.counters[b], 1);
                 last_flag[1] = ((uint32_t)old == j_last - j_first);
             }
             if (!consumers_sync()) return;
             if (last_flag[1]) {
-                __threadfence();
+                // all contributors' parts are loaded together (one L2 round
+                // trip for up to kPar of them), then added in CTA order; this
+                // CTA's own part is still in registers
+                constexpr int kPar = MT <= 2 ? 8 : 2;
+                float own[MT][4];
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) sum[mt][e] = 0.0f;
-                for (uint32_t j = j_first; j <= j_last; ++j) {
-                    const uint32_t sj = (range_start(j, p.T, p.G) / KB == b) ? 2 * j : 2 * j + 1;
-                    const float *src = p.partials + (int64_t)sj * C::kPartialFloats;
-                    float part[MT][4];
+                    for (int e = 0; e < 4; ++e) {
+                        own[mt][e] = sum[mt][e];
+                        sum[mt][e] = 0.0f;
+                    }
+                for (uint32_t j0 = j_first; j0 <= j_last; j0 += kPar) {
+                    float part[kPar][MT][4];
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
+                    for (int u = 0; u < kPar; ++u) {
+                        const uint32_t j = j0 + u;
+                        if (j <= j_last && j != cta) {
+                            const uint32_t sj = (range_start(j, p.T, p.G) / KB == b) ? 2 * j : 2 * j + 1;
+                            const float *src = p.partials + (int64_t)sj * C::kPartialFloats;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            part[mt][e] = __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
+                            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
+                                for (int e = 0; e < 4; ++e)
+                                    part[u][mt][e] = __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
+                        } else {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) sum[mt][e] += part[mt][e];
+                            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) part[u][mt][e] = own[mt][e];
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < kPar; ++u) {
+                        if (j0 + u <= j_last) {
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) sum[mt][e] += part[u][mt][e];
+                        }
+                    }
                 }
                 store_y<MT>(p, b, warp, lane, sum);
                 if (threadIdx.x == 0) p.counters[b] = 0;
