@@ -123,10 +123,12 @@ int w8_unpack(const uint8_t *packed, int64_t K, int64_t N, int8_t *q, void *stre
 
 /*
  * w8a16_workspace_bytes -- device scratch w8a16_linear needs for this shape
- * on the CURRENT device (it depends on the SM count).  0 means none.  The
- * weight-streaming path (M <= 64) splits the reduction over K across
- * thread blocks and needs room for fp32 partial sums (a fixed 64 KB per
- * multiprocessor) plus one int32 counter per 128 output channels.
+ * on the CURRENT device (it depends on the SM count); 0 only for an empty
+ * shape or when no device is usable.  Both kernels split the reduction over
+ * K across thread blocks where the output alone would not fill the GPU and
+ * need room for fp32 partial sums (a fixed 256 KB per multiprocessor, the
+ * same for every shape) plus int32 counters (the larger of one per 128
+ * output channels and two per multiprocessor).
  */
 size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
 
@@ -158,7 +160,10 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
  * split-K kernel on the legacy tensor-core path (HBM-bound up to about 32
  * tokens); larger M runs a tcgen05 tensor-core kernel on pairs of SMs
  * (clusters of two thread blocks) with the widened weight tile held in
- * tensor memory.
+ * tensor memory, whole 256 x 256 output tiles per pair where they fill
+ * the GPU and a K split over all pairs for the tiles that do not.  Both
+ * add a tile's partial sums in a fixed order: results are the same on
+ * every call.
  * Accuracy: |Y - Y_exact| <= 2^-9 |Y_exact| + 1e-3 rms(Y_exact).
  * Errors: W8_ERR_NULL, W8_ERR_SHAPE, W8_ERR_ALIGN, W8_ERR_WORKSPACE,
  *         W8_ERR_ALIAS, W8_ERR_DEVICE, W8_ERR_CUDA.

@@ -45,6 +45,7 @@ enum WaitSite : unsigned {
     SITE_P2_DEMPTY = 0x46,
     SITE_P2_DFULL = 0x47,
     SITE_P2_DRAIN = 0x48,
+    SITE_P2_FIX = 0x49,
     SITE_SELFTEST = 0xEE,
 };
 
@@ -396,6 +397,20 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Barrier over nthreads threads that also returns whether pred holds in
+// all of them (so that a group of warps agrees on giving up a wait).
+__device__ __forceinline__ bool named_bar_all(uint32_t id, uint32_t nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
 }
 
 // ---------------------------------------------------------------- int8 widening

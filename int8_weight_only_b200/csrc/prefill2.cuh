@@ -30,6 +30,16 @@
 //   warps 8-15  epilogue: drain this CTA's 128 accumulator lanes, release
 //               the accumulator on the first CTA's barrier, scale, store.
 //   warp 2      tensor-memory allocation for the pair.
+//
+// Schedule.  The pairs are persistent.  Whole tiles go round robin over the
+// pairs for all but the last wave ("data-parallel" part); the 256-wide K
+// steps of the tiles that remain are then split evenly over all pairs
+// (a stream-K split), so that the work per pair differs by at most one K
+// step whatever the tile count.  A pair's share of a tile ends in one of
+// two fp32 partial-sum slots of the workspace; the pair that brings a
+// tile's arrival count to its number of contributors adds the partial sums
+// in K order (a fixed order: results do not depend on timing), scales and
+// stores the tile.  No pair ever waits for another.
 #pragma once
 
 #include "common.cuh"
@@ -67,18 +77,80 @@ static_assert(kXBox % 1024 == 0 && kWBytes % 1024 == 0, "stage alignment");
 static_assert(kAcol0 + 32 * kKStep * kABuf <= kTmemCols, "tensor memory budget");
 static_assert(kSmemBytes <= 227 * 1024 - 512, "shared memory budget");
 
+// fp32 partial sums of one CTA's share of a pair tile: [256 tokens][128 channels]
+constexpr int kPartFloats = kBT * kBNc;
+
+
 struct Params {
     const uint8_t *packed;
     const uint16_t *scales;
     const uint16_t *bias;   // may be null
     uint16_t *Y;
+    float *partials;        // [pairs][2 slots][2 CTAs][kPartFloats]
+    int *counters;          // [stream-K tiles][2 CTAs], zero between calls
     int M;
     int64_t N;
     int NB;        // ceil(N/128): packed channel blocks
     int KB;        // ceil(K/64)
     int KS;        // ceil(KB/4): 256-wide K steps
     int TT;        // token tiles = ceil(M/256)
-    int64_t tiles; // ceil(NB/2) * TT pair tiles
+    int tiles;     // ceil(NB/2) * TT pair tiles
+    int dp_tiles;  // tiles [0, dp_tiles) run whole, round robin
+    int sk_iters;  // K steps of tiles [dp_tiles, tiles), split evenly
+};
+
+// First stream-K step of pair q (steps numbered from tile dp_tiles' first).
+// The host keeps tiles, sk_iters and sk_iters x pairs below 2^31.
+__device__ __forceinline__ int sk_begin(int q, int pairs, int iters) {
+    return (int)((int64_t)q * iters / pairs);
+}
+// The pair whose share holds stream-K step it: the largest q with
+// sk_begin(q) <= it.  Every pair has at least one step (iters >= pairs).
+__device__ __forceinline__ int sk_owner(int it, int pairs, int iters) {
+    return (int)(((int64_t)(it + 1) * pairs - 1) / iters);
+}
+// Partial-sum slot that pair q uses for stream-K tile t: 0 for the tile its
+// share starts in, 1 for the tile it ends in (every tile between is whole).
+__device__ __forceinline__ int sk_slot(int q, int t, int pairs, int iters, int KS) {
+    return sk_begin(q, pairs, iters) / KS == t ? 0 : 1;
+}
+
+// One segment of a pair's work: K steps [ks0, ks1) of one pair tile.
+struct Seg {
+    int tile;
+    int ks0, ks1;
+    int slot;     // -1: the whole tile; else the partial-sum slot
+    bool final;   // the pair's last segment
+};
+
+struct Sched {
+    int tile, pairs, dp_tiles, it, it_end, it_first, KS;
+    __device__ Sched(int q, int npairs, int dp, int sk_iters, int ks)
+        : tile(q), pairs(npairs), dp_tiles(dp), KS(ks) {
+        it_first = it = sk_iters > 0 ? sk_begin(q, npairs, sk_iters) : 0;
+        it_end = sk_iters > 0 ? sk_begin(q + 1, npairs, sk_iters) : 0;
+    }
+    __device__ bool more() const { return tile < dp_tiles || it < it_end; }
+    __device__ bool next(Seg &s) {
+        if (tile < dp_tiles) {
+            s.tile = tile;
+            s.ks0 = 0;
+            s.ks1 = KS;
+            s.slot = -1;
+            tile += pairs;
+        } else if (it < it_end) {
+            const int t = it / KS;
+            s.tile = dp_tiles + t;
+            s.ks0 = it - t * KS;
+            s.ks1 = min(KS, s.ks0 + (it_end - it));
+            s.slot = (s.ks0 == 0 && s.ks1 == KS) ? -1 : (t == it_first / KS ? 0 : 1);
+            it += s.ks1 - s.ks0;
+        } else {
+            return false;
+        }
+        s.final = !more();
+        return true;
+    }
 };
 
 struct Ring {
@@ -92,9 +164,111 @@ struct Ring {
     }
 };
 
+// The epilogue's part in one share of a stream-K tile (all kEpiWarps
+// warps call it together, once the share's accumulator is complete):
+// publish the share's fp32 partial sums, count it, and when it is the
+// tile's last share to be counted add all shares in K order, scale and
+// store Y.  A pair on its last segment keeps its accumulator (nothing
+// waits for it) and, if every other share is already counted, completes
+// the tile from tensor memory without publishing its own.
+__device__ __forceinline__ void stream_k_share(float *partials, int *counters, uint16_t *Y, const int M,
+                                               const int64_t N, const int dp_tiles, const int sk_iters,
+                                               const int KS, const Seg &sg, const int pair0, const int pstep,
+                                               const uint32_t tmem, const uint32_t rank, const int warp,
+                                               const int lane, int *fix_last, const uint32_t d_empty_leader,
+                                               const float sc, const float bi, const bool n_ok, const int64_t n,
+                                               const int tb) {
+    const int q4 = warp & 3;
+    const int half = (warp - 8) >> 2;
+    const int r = 32 * q4 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16) + 128 * half;
+    const int m0 = tb * kBT + 128 * half;
+    const int t = sg.tile - dp_tiles;
+    const int j_first = sk_owner(t * KS, pstep, sk_iters);
+    const int j_last = sk_owner(t * KS + KS - 1, pstep, sk_iters);
+    const int others = j_last - j_first;
+    int *cnt = counters + t * 2 + rank;
+    const int64_t elem = 128 * half * kBNc + r;   // this thread's first element of a share
+    auto part_of = [&](int j) -> float * {
+        const int slot = sk_slot(j, t, pstep, sk_iters, KS);
+        return partials + (int64_t)((j * 2 + slot) * 2 + (int)rank) * kPartFloats + elem;
+    };
+    if (sg.final) {
+        if (warp == 8 && lane == 0) *fix_last = ld_acquire_gpu(cnt) == others;
+        named_bar_sync(1, 32 * kEpiWarps);
+    }
+    const bool publish = !(sg.final && *fix_last);
+    if (publish) {
+        float *mine = part_of(pair0);
+#pragma unroll
+        for (int cchunk = 0; cchunk < 4; ++cchunk) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(lane_addr + 32 * cchunk, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) __stcg(mine + (32 * cchunk + i) * kBNc, __uint_as_float(v[i]));
+        }
+    }
+    if (!sg.final) {   // more work follows: free the accumulator now
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(d_empty_leader);
+    }
+    if (publish) {
+        named_bar_sync(1, 32 * kEpiWarps);   // every part of this CTA is written
+        if (warp == 8 && lane == 0) {
+            // release (with the barrier above) and acquire in one atomic
+            const int last = atomic_add_acq_rel_gpu(cnt, 1) == others;
+            if (last) *cnt = 0;   // every share is counted: ready for the next call
+            *fix_last = last;
+        }
+        named_bar_sync(1, 32 * kEpiWarps);
+    } else if (warp == 8 && lane == 0) {
+        *cnt = 0;
+    }
+    if (*fix_last) {
+#pragma unroll 1
+        for (int cchunk = 0; cchunk < 4; ++cchunk) {
+            float acc[32];
+#pragma unroll 1
+            for (int j = j_first; j <= j_last; ++j) {
+                uint32_t v[32];
+                if (j == pair0 && sg.final) {
+                    tmem_ld_32x32b_x32(lane_addr + 32 * cchunk, v);
+                    tmem_wait_ld();
+                } else {
+                    const float *src = part_of(j) + 32 * cchunk * kBNc;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__ldcg(src + i * kBNc));
+                }
+                if (j == j_first) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(v[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] += __uint_as_float(v[i]);
+                }
+            }
+            if (n_ok) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int m = m0 + 32 * cchunk + i;
+                    if (m < M) Y[(int64_t)m * N + n] = __half_as_ushort(__float2half_rn(fmaf(acc[i], sc, bi)));
+                }
+            }
+        }
+    }
+    if (sg.final) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(d_empty_leader);
+    }
+}
+
 // grid = 2 x pairs CTAs, cluster dims (2, 1, 1), kThreads threads,
 // kSmemBytes dynamic shared memory.  tmap_x: X [M, K] fp16, box {64, 128},
 // 128-byte swizzle.
+template <bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -107,12 +281,13 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     __shared__ uint64_t a_full[kABuf], a_empty[kABuf];
     __shared__ uint64_t d_full, d_empty, drain;
     __shared__ uint32_t tmem_base_sh;
+    __shared__ int fix_last;       // this CTA completes the current tile
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();     // 0: issues the pair MMAs
-    const int64_t pair0 = blockIdx.x >> 1;
-    const int64_t pstep = gridDim.x >> 1;
+    const int pair0 = blockIdx.x >> 1;
+    const int pstep = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kWStages; ++i) {
@@ -151,11 +326,13 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             Ring r;
             int issued = 0;
             bool ok = true;
-            for (int64_t pt = pair0; pt < p.tiles && ok; pt += pstep) {
-                const int64_t blk = (pt / p.TT) * 2 + rank;
+            Sched sched(pair0, pstep, p.dp_tiles, p.sk_iters, p.KS);
+            Seg sg;
+            while (ok && sched.next(sg)) {
+                const int64_t blk = (sg.tile / p.TT) * 2 + rank;
                 const bool valid = blk < p.NB;
                 const uint8_t *wsrc = p.packed + blk * p.KB * (int64_t)kWTile;
-                for (int ks = 0; ks < p.KS; ++ks) {
+                for (int ks = sg.ks0; ks < sg.ks1; ++ks) {
                     const int cnt = min(kKStep, p.KB - kKStep * ks);   // tiles in this step
                     if (!mbar_wait(&w_empty[r.s], r.ph ^ 1u, SITE_P2_WEMPTY)) { ok = false; break; }
                     if (valid) {
@@ -180,9 +357,11 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             Ring r;
             int issued = 0;
             bool ok = true;
-            for (int64_t pt = pair0; pt < p.tiles && ok; pt += pstep) {
-                const int tb = (int)(pt % p.TT);
-                for (int ks = 0; ks < p.KS; ++ks) {
+            Sched sched(pair0, pstep, p.dp_tiles, p.sk_iters, p.KS);
+            Seg sg;
+            while (ok && sched.next(sg)) {
+                const int tb = (int)(sg.tile % p.TT);
+                for (int ks = sg.ks0; ks < sg.ks1; ++ks) {
                     const int cnt = min(kKStep, p.KB - kKStep * ks);
                     if (!mbar_wait(&x_empty[r.s], r.ph ^ 1u, SITE_P2_XEMPTY)) { ok = false; break; }
                     if (rank == 0) mbar_arrive_expect_tx(&x_full[r.s], 2 * cnt * kXBox);
@@ -210,10 +389,12 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             Ring xr, ar;
             int it = 0;
             bool ok = true;
-            for (int64_t pt = pair0; pt < p.tiles && ok; pt += pstep, ++it) {
+            Sched sched(pair0, pstep, p.dp_tiles, p.sk_iters, p.KS);
+            Seg sg;
+            for (; ok && sched.next(sg); ++it) {
                 if (!mbar_wait(&d_empty, (it & 1) ^ 1u, SITE_P2_DEMPTY)) { ok = false; break; }
                 tc_fence_after();
-                for (int ks = 0; ks < p.KS; ++ks) {
+                for (int ks = sg.ks0; ks < sg.ks1; ++ks) {
                     const int cnt = min(kKStep, p.KB - kKStep * ks);
                     if (!mbar_wait(&x_full[xr.s], xr.ph, SITE_P2_XFULL)) { ok = false; break; }
                     if (!mbar_wait(&a_full[ar.s], ar.ph, SITE_P2_AFULL)) { ok = false; break; }
@@ -225,7 +406,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                         for (int j = 0; j < 4; ++j)
                             tc_mma_ts_f16_pair(tmem, a_tmem + 32 * t + 8 * j,
                                                smem_desc_kmajor_sw128(x_addr + t * kXBox + 32 * j), kIdesc,
-                                               (ks | t | j) != 0);
+                                               ((ks - sg.ks0) | t | j) != 0);
                     }
                     tc_commit_pair_mc(&x_empty[xr.s], kBoth);
                     tc_commit_pair_mc(&a_empty[ar.s], kBoth);
@@ -247,9 +428,11 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
         Ring wr, ar;
         bool ok = true;
-        for (int64_t pt = pair0; pt < p.tiles && ok; pt += pstep) {
-            const bool valid = (pt / p.TT) * 2 + rank < p.NB;
-            for (int ks = 0; ks < p.KS; ++ks) {
+        Sched sched(pair0, pstep, p.dp_tiles, p.sk_iters, p.KS);
+        Seg sg;
+        while (ok && sched.next(sg)) {
+            const bool valid = (sg.tile / p.TT) * 2 + rank < p.NB;
+            for (int ks = sg.ks0; ks < sg.ks1; ++ks) {
                 const int cnt = min(kKStep, p.KB - kKStep * ks);
                 if (!warp_all(mbar_wait(&w_full[wr.s], wr.ph, SITE_P2_WFULL))) { ok = false; break; }
                 uint4 c[kKStep][4];
@@ -298,39 +481,53 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         const int r = 32 * q4 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16) + 128 * half;
         int it = 0;
-        for (int64_t pt = pair0; pt < p.tiles; pt += pstep, ++it) {
-            if (!warp_all(mbar_wait(&d_full, it & 1, SITE_P2_DFULL))) break;
+        Sched sched(pair0, pstep, p.dp_tiles, p.sk_iters, p.KS);
+        Seg sg;
+        for (; sched.next(sg); ++it) {
+            const bool got = warp_all(mbar_wait(&d_full, it & 1, SITE_P2_DFULL));
+            if constexpr (kSplit) {
+                // all epilogue warps give up together: the stream-K share
+                // below has barriers over all of them
+                if (!named_bar_all(1, 32 * kEpiWarps, got)) break;
+            } else {
+                if (!got) break;
+            }
             tc_fence_after();
-            const int64_t blk = (pt / p.TT) * 2 + rank;
-            const int tb = (int)(pt % p.TT);
+            const int64_t blk = (sg.tile / p.TT) * 2 + rank;
+            const int tb = (int)(sg.tile % p.TT);
             const int64_t n = blk * kBNc + r;
             const bool n_ok = n < p.N;
             const float sc = n_ok ? __half2float(__ushort_as_half(p.scales[n])) : 0.0f;
             const float bi = (n_ok && p.bias) ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
-            uint32_t y2[64];
-#pragma unroll
-            for (int cchunk = 0; cchunk < 4; ++cchunk) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(lane_addr + 32 * cchunk, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const __half2 hv = __floats2half2_rn(fmaf(__uint_as_float(v[2 * i]), sc, bi),
-                                                         fmaf(__uint_as_float(v[2 * i + 1]), sc, bi));
-                    y2[16 * cchunk + i] = *reinterpret_cast<const uint32_t *>(&hv);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(leader(&d_empty));
-            if (n_ok) {
+            if (sg.slot < 0) {
                 const int m0 = tb * kBT + 128 * half;
+                uint32_t y2[64];
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const int m = m0 + 2 * i;
-                    if (m < p.M) p.Y[(int64_t)m * p.N + n] = (uint16_t)(y2[i] & 0xFFFFu);
-                    if (m + 1 < p.M) p.Y[(int64_t)(m + 1) * p.N + n] = (uint16_t)(y2[i] >> 16);
+                for (int cchunk = 0; cchunk < 4; ++cchunk) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(lane_addr + 32 * cchunk, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const __half2 hv = __floats2half2_rn(fmaf(__uint_as_float(v[2 * i]), sc, bi),
+                                                             fmaf(__uint_as_float(v[2 * i + 1]), sc, bi));
+                        y2[16 * cchunk + i] = *reinterpret_cast<const uint32_t *>(&hv);
+                    }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(leader(&d_empty));
+                if (n_ok) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const int m = m0 + 2 * i;
+                        if (m < p.M) p.Y[(int64_t)m * p.N + n] = (uint16_t)(y2[i] & 0xFFFFu);
+                        if (m + 1 < p.M) p.Y[(int64_t)(m + 1) * p.N + n] = (uint16_t)(y2[i] >> 16);
+                    }
+                }
+            } else if constexpr (kSplit) {
+                stream_k_share(p.partials, p.counters, p.Y, p.M, p.N, p.dp_tiles, p.sk_iters, p.KS, sg, pair0,
+                               pstep, tmem, rank, warp, lane, &fix_last, leader(&d_empty), sc, bi, n_ok, n, tb);
             }
         }
     }

@@ -66,7 +66,11 @@ int device_info(DeviceInfo **out) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          decode::Cfg<8>::kSmemBytes);
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(prefill2::prefill2_kernel,
+                e = cudaFuncSetAttribute(prefill2::prefill2_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         prefill2::kSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(prefill2::prefill2_kernel<true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          prefill2::kSmemBytes);
             if (e == cudaSuccess)
@@ -215,7 +219,8 @@ int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t 
 
 // Tensor-core linear for M > 64 on CTA pairs (prefill2.cuh).
 int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
-                    const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N, cudaStream_t st) {
+                    const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N, float *partials,
+                    int *counters, cudaStream_t st) {
     CUtensorMap map;
     int rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
                          prefill2::kBTc, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -225,13 +230,18 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
     p.scales = scales;
     p.bias = bias;
     p.Y = Y;
+    p.partials = partials;
+    p.counters = counters;
     p.M = (int)M;
     p.N = N;
     p.NB = (int)cdiv(N, 128);
     p.KB = (int)cdiv(K, 64);
     p.KS = (int)cdiv(p.KB, prefill2::kKStep);
     p.TT = (int)cdiv(M, prefill2::kBT);
-    p.tiles = cdiv(p.NB, 2) * p.TT;
+    const int64_t tiles = cdiv(p.NB, 2) * p.TT;
+    // 32-bit work counts (a 2^31-tile output would not fit in device memory)
+    if (tiles >= INT32_MAX / 2 || (int64_t)p.KS * 2 * d->sms >= INT32_MAX) return W8_ERR_SHAPE;
+    p.tiles = (int)tiles;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(prefill2::kThreads, 1, 1);
     cfg.dynamicSmemBytes = prefill2::kSmemBytes;
@@ -249,7 +259,7 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
         if (d->pairs == 0) {
             cfg.gridDim = dim3((unsigned)d->sms, 1, 1);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, prefill2::prefill2_kernel, &cfg) != cudaSuccess || n < 1) {
+            if (cudaOccupancyMaxActiveClusters(&n, prefill2::prefill2_kernel<false>, &cfg) != cudaSuccess || n < 1) {
                 cudaGetLastError();
                 n = d->sms / 2;
             }
@@ -257,9 +267,42 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
         }
         resident = d->pairs;
     }
-    const int64_t pairs = std::min<int64_t>(p.tiles, resident);
+    // Schedule (prefill2.cuh).  Whole tiles round robin over the pairs,
+    // unless splitting the last waves' K steps over all pairs saves at least
+    // kSplitMinSteps 256-wide K steps per pair: a split tile's fix-up
+    // (partial sums written, counted, read back and added) costs 20-40 us
+    // on the critical path, measured, against about 1.65 us per K step.
+    // That holds for long K with few tiles (e.g. 13696 x 4096 with M up to
+    // 512).  The pair count never exceeds half the SMs (the workspace's
+    // partial-sum slots).
+    constexpr int64_t kSplitMinSteps = 24;
+    const int P = std::max(1, std::min(resident, d->sms / 2));
+    int pairs = std::min(P, p.tiles), sk_tiles = 0, split_pairs = P;
+    if (p.tiles >= P) {
+        if (p.tiles % P != 0 && p.KS > 1) sk_tiles = P + p.tiles % P;
+    } else if (p.KS > 1) {
+        sk_tiles = p.tiles;
+        split_pairs = (int)std::min<int64_t>(P, (int64_t)p.tiles * p.KS);   // at least one K step each
+    }
+    bool split = false;
+    if (sk_tiles > 0) {
+        const int64_t whole_steps = cdiv(p.tiles, P) * p.KS;
+        const int64_t split_steps =
+            (int64_t)((p.tiles - sk_tiles) / P) * p.KS + cdiv((int64_t)sk_tiles * p.KS, split_pairs);
+        split = whole_steps - split_steps >= kSplitMinSteps;
+    }
+    if (split) {
+        pairs = split_pairs;
+        p.dp_tiles = p.tiles - sk_tiles;
+        p.sk_iters = sk_tiles * p.KS;   // < 2 P KS
+    } else {
+        p.dp_tiles = p.tiles;
+        p.sk_iters = 0;
+    }
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-    if (cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel, map, p) != cudaSuccess) {
+    const cudaError_t e = split ? cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<true>, map, p)
+                                : cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<false>, map, p);
+    if (e != cudaSuccess) {
         cudaGetLastError();
         return W8_ERR_CUDA;
     }
@@ -356,25 +399,32 @@ int w8_unpack(const uint8_t *packed, int64_t K, int64_t N, int8_t *q, void *stre
 // Decode split: one CTA per SM (never more CTAs than tiles).
 static int decode_grid(int sms, int64_t T) { return (int)std::max<int64_t>(1, std::min<int64_t>(T, sms)); }
 
-// Decode workspace: [partials: 2 slots per SM][counters: one int32 per 128
-// channels].  The partial area has the same size for every shape on a
-// device, so the counters always start at the same offset: a workspace that
-// served one shape (and was left with zero counters) serves any other.
+// Workspace: [fp32 partial sums][int32 counters].  The partial area is the
+// larger of the two kernels' needs -- decode: 2 slots per SM; prefill: 2
+// slots per CTA pair, each a 256-token x 256-channel tile -- and has the
+// same size for every shape on a device, so the counters always start at
+// the same offset: a workspace that served one shape (and was left with
+// zero counters) serves any other.  Counters: one per 128 channels
+// (decode) or two per stream-K tile, fewer than 2 x SMs (prefill).
 static size_t decode_partials_bytes(int sms) {
     return (size_t)2 * sms * decode::kMaxPartialFloats * sizeof(float);
 }
 
-static size_t decode_workspace(int sms, int64_t K, int64_t N) {
-    (void)K;
-    const int64_t NB = cdiv(N, 128);
-    return decode_partials_bytes(sms) + (size_t)cdiv(NB * 4, 256) * 256;
+static size_t partial_area_bytes(int sms) {
+    const size_t pre = (size_t)(sms / 2) * 4 * prefill2::kPartFloats * sizeof(float);
+    return std::max(decode_partials_bytes(sms), pre);
+}
+
+static size_t workspace_total(int sms, int64_t N) {
+    const int64_t counters = std::max<int64_t>(cdiv(N, 128), 2 * (int64_t)sms);
+    return partial_area_bytes(sms) + (size_t)cdiv(counters * 4, 256) * 256;
 }
 
 size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N) {
-    if (M < 1 || M > decode::kMaxTokens || K < 1 || N < 1) return 0;
+    if (M < 1 || K < 1 || N < 1) return 0;
     DeviceInfo *d = nullptr;
     if (device_info(&d) != W8_OK) return 0;
-    return decode_workspace(d->sms, K, N);
+    return workspace_total(d->sms, N);
 }
 
 int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
@@ -401,11 +451,14 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
     const int KB = (int)cdiv(K, 64);
     const int64_t NB = cdiv(N, 128);
 
+    const size_t need = workspace_total(d->sms, N);
+    if (!workspace || workspace_bytes < need) return W8_ERR_WORKSPACE;
+    if (overlap(workspace, need, Y, ybytes) || overlap(workspace, need, X, (size_t)M * K * 2))
+        return W8_ERR_ALIAS;
+    float *partials = static_cast<float *>(workspace);
+    int *counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + partial_area_bytes(d->sms));
+
     if (M <= decode::kMaxTokens) {
-        const size_t need = decode_workspace(d->sms, K, N);
-        if (!workspace || workspace_bytes < need) return W8_ERR_WORKSPACE;
-        if (overlap(workspace, need, Y, ybytes) || overlap(workspace, need, X, (size_t)M * K * 2))
-            return W8_ERR_ALIAS;
         const int MT = M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8;
         CUtensorMap map;
         rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
@@ -416,9 +469,8 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
         p.scales = scales;
         p.bias = bias;
         p.Y = Y;
-        p.partials = static_cast<float *>(workspace);
-        p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) +
-                                             decode_partials_bytes(d->sms));
+        p.partials = partials;
+        p.counters = counters;
         p.M = (int)M;
         p.N = N;
         p.KB = KB;
@@ -435,7 +487,7 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
         }
     }
 
-    return launch_prefill2(d, X, packed, scales, bias, Y, M, K, N, st);
+    return launch_prefill2(d, X, packed, scales, bias, Y, M, K, N, partials, counters, st);
 }
 
 // ---------------------------------------------------------------- diagnostics

@@ -51,6 +51,59 @@ def test_prefill_matches_oracle(M, K, N):
     _check_full(M, K, N, 3000 + K + N + M, bias=(M % 2 == 0))
 
 
+def _sampled_blocks(M, K, N, tid, bias=True, per_block=2, seed=3):
+    """GPU pipeline on the whole problem; the oracle on `per_block` channels
+    of every 128-channel block (all tokens)."""
+    W, X, b = _case(M, K, N, tid, bias)
+    qg, sg, Yg = gpu_pipeline(W, X, b)
+    rng = np.random.default_rng(seed)
+    cols = np.sort(np.concatenate([blk * 128 + rng.choice(min(128, N - blk * 128), per_block, replace=False)
+                                   for blk in range((N + 127) // 128)]))
+    qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
+    assert np.array_equal(qg[:, cols], qo)
+    assert_close(Yg[:, cols], oracle.linear(X, qo, so, None if b is None else b[cols]), f"M={M} K={K} N={N}")
+    return Yg
+
+
+def test_prefill_k_split_one_step_shares():
+    # 2 pair tiles of 32 K steps: the K steps are split over 64 pairs, one
+    # step each, and every tile is summed from 32 partial sums; full check
+    _check_full(129, 8192, 512, 3900, bias=True)
+
+
+def test_prefill_k_split_shares_cross_tiles():
+    # 16 pair tiles of 32 K steps over 74 pairs: shares of 6 or 7 steps start
+    # and end inside tiles (both partial-sum slots in use)
+    _sampled_blocks(300, 8192, 2048, 3910)
+
+
+def test_prefill_whole_wave_then_k_split():
+    # 150 pair tiles of 32 K steps: one wave of whole tiles, then the K steps
+    # of the last 76 tiles split over all pairs
+    _sampled_blocks(3800, 8192, 2560, 3920, per_block=1)
+
+
+def test_prefill_k_split_deterministic():
+    # the split tiles' partial sums are added in K order whatever the order
+    # in which the pairs finish: repeated calls agree bit for bit
+    torch = pytest.importorskip("torch")
+    m = w8()
+    W, X, b = _case(300, 8192, 2048, 3930)
+    q, s = m.quantize(to_gpu(W))
+    packed = m.prepack(q)
+    Xg, bg = to_gpu(X), to_gpu(b)
+    Y1 = to_np(m.linear(Xg, packed, s, bg))
+    for _ in range(3):
+        Y2 = to_np(m.linear(Xg, packed, s, bg))
+        assert np.array_equal(Y1.view(np.uint16), Y2.view(np.uint16))
+
+
+def test_prefill_whole_waves_ragged_tail_sampled():
+    # 190 pair tiles of 2 K steps: three waves of whole tiles, the last one
+    # partly filled
+    _sampled_blocks(1280, 512, 9728, 3950)
+
+
 def test_tiny_workload_both_paths():
     # 4 x 256 activations, 256 x 512 weight (the smallest workload), then the
     # same weight through the tensor-core path with 4 copies of X stacked
@@ -109,9 +162,11 @@ def test_deterministic_across_calls():
 
 def test_workspace_reused_across_shapes():
     # the split-K counters are reset by each call, so one workspace serves
-    # calls of different shapes and token counts back to back
+    # calls of different shapes and token counts back to back, weight
+    # streaming and tensor-core paths alike
     for (M, K, N) in [(1, 4096, 512), (3, 64, 8), (16, 1000, 1032), (64, 2048, 4104), (1, 4096, 512),
-                      (40, 4096, 27392), (9, 13696, 264)]:
+                      (300, 8192, 2048), (40, 4096, 27392), (129, 8192, 512), (9, 13696, 264),
+                      (129, 8192, 512)]:
         _check_full(M, K, N, 3700 + K + N)
 
 
@@ -127,8 +182,9 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(m.W8Error) as e:
         m.linear(to_gpu(X), packed, s, workspace=ws)
     assert e.value.status == -5
-    assert m.workspace_bytes(64, 256, 512) > 0
-    assert m.workspace_bytes(65, 256, 512) == 0
+    # one layout for every token count: the K-split partial sums of both kernels
+    assert m.workspace_bytes(65, 256, 512) == m.workspace_bytes(64, 256, 512) > 0
+    assert m.workspace_bytes(0, 256, 512) == 0
 
 
 def test_empty_batch():
