@@ -60,8 +60,12 @@ class Oracle:
         lib.oracle_quantize_f32.argtypes = [vp, i64, i64, vp, vp, vp]
         lib.oracle_quantize_f16.argtypes = [vp, i64, i64, vp, vp, vp]
         lib.oracle_linear.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
+        lib.oracle_quantize_asym_f32.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        lib.oracle_quantize_asym_f16.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        lib.oracle_linear_asym.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
         for f in ("oracle_f32_to_f16_array", "oracle_f16_to_f32_array",
-                  "oracle_quantize_f32", "oracle_quantize_f16", "oracle_linear"):
+                  "oracle_quantize_f32", "oracle_quantize_f16", "oracle_linear",
+                  "oracle_quantize_asym_f32", "oracle_quantize_asym_f16", "oracle_linear_asym"):
             getattr(lib, f).restype = None
         self.lib = lib
         self.path = so_path
@@ -121,6 +125,48 @@ class Oracle:
         return Y
 
 
+    def quantize_asym(self, W: np.ndarray):
+        """Per-output-channel asymmetric (affine) int8 quantization.
+
+        W: [K, N] float32 or float16.  Returns (q int8 [K, N], scales
+        float16 [N], zeros int8 [N]); a weight is dequantized as
+        (q - zero) * scale.
+        """
+        if W.ndim != 2:
+            raise ValueError("W must be 2-D [K, N]")
+        K, N = W.shape
+        q = np.empty((K, N), dtype=np.int8)
+        s = np.empty(N, dtype=np.uint16)
+        z = np.empty(N, dtype=np.int8)
+        buf = np.empty(max(K, 1), dtype=np.float32)
+        if W.dtype == np.float32:
+            Wc = np.ascontiguousarray(W)
+            self.lib.oracle_quantize_asym_f32(_ptr(Wc), K, N, _ptr(q), _ptr(s), _ptr(z), _ptr(buf))
+        elif W.dtype == np.float16:
+            Wc = np.ascontiguousarray(W).view(np.uint16)
+            self.lib.oracle_quantize_asym_f16(_ptr(Wc), K, N, _ptr(q), _ptr(s), _ptr(z), _ptr(buf))
+        else:
+            raise TypeError("W must be float32 or float16")
+        return q, s.view(np.float16), z
+
+    def linear_asym(self, X, q, scales, zeros, bias=None) -> np.ndarray:
+        """Y = X . ((q - zeros) o scales) (+ bias) in fp64 (not rounded)."""
+        M, K = X.shape
+        K2, N = q.shape
+        if K2 != K or scales.shape != (N,) or zeros.shape != (N,):
+            raise ValueError("shape mismatch")
+        Xc = np.ascontiguousarray(X, dtype=np.float16).view(np.uint16)
+        qc = np.ascontiguousarray(q, dtype=np.int8)
+        sc = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
+        zc = np.ascontiguousarray(zeros, dtype=np.int8)
+        bc = None if bias is None else np.ascontiguousarray(bias, dtype=np.float16).view(np.uint16)
+        Y = np.empty((M, N), dtype=np.float64)
+        acc = np.empty(max(N, 1), dtype=np.float64)
+        self.lib.oracle_linear_asym(_ptr(Xc), _ptr(qc), _ptr(sc), _ptr(zc),
+                                    None if bc is None else _ptr(bc), M, K, N, _ptr(Y), _ptr(acc))
+        return Y
+
+
 def default() -> Oracle:
     global _default
     with _lock:
@@ -143,6 +189,14 @@ def quantize(W):
 
 def linear(X, q, scales, bias=None):
     return default().linear(X, q, scales, bias)
+
+
+def quantize_asym(W):
+    return default().quantize_asym(W)
+
+
+def linear_asym(X, q, scales, zeros, bias=None):
+    return default().linear_asym(X, q, scales, zeros, bias)
 
 
 def tolerance_ok(y_test: np.ndarray, y_ref: np.ndarray):

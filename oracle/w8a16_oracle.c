@@ -225,6 +225,124 @@ void oracle_linear(const uint16_t *X, const int8_t *q, const uint16_t *scales,
     }
 }
 
+/* ---------------------------------------------------------------------
+ * Asymmetric (affine) per-output-channel int8 quantization -- the variant
+ * the LightSeq 2020 slides set against the symmetric one (slide
+ * "quantization: clipping + symmetric": a weight is (i - z) S, and the
+ * product of two such values expands into four integer terms), with the
+ * range, scale and zero point of the integer-arithmetic quantization paper
+ * those slides cite (arXiv 1712.05877, section 2):
+ *   lo = min(0, min_k W), hi = max(0, max_k W)   (0 stays representable)
+ *   S  = fp16_rne( fp32(hi - lo) / 255 )          (256 levels, -128..127)
+ *   z  = clamp( rne( -128 - lo / S ), -128, 127 )
+ *   q  = clamp( rne( W / S ) + z, -128, 127 )
+ * every operation in IEEE fp32 with S the stored fp16 value widened; an
+ * all-zero column has S = 0, z = 0 and q = 0.  Dequantized: (q - z) S.
+ * ------------------------------------------------------------------- */
+
+static float clampf_range(float v, float lo, float hi)
+{
+    if (v < lo) {
+        return lo;
+    }
+    if (v > hi) {
+        return hi;
+    }
+    return v;
+}
+
+static void quantize_column_asym(const float *col_vals, int64_t K, int8_t *q_col,
+                                 int64_t N, uint16_t *scale_out, int8_t *zero_out)
+{
+    float lo = 0.0f, hi = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        if (col_vals[k] < lo) {
+            lo = col_vals[k];
+        }
+        if (col_vals[k] > hi) {
+            hi = col_vals[k];
+        }
+    }
+    float range = hi - lo;                       /* IEEE fp32 subtraction */
+    uint16_t s16 = oracle_f32_to_f16(range / 255.0f);
+    float s = oracle_f16_to_f32(s16);
+    int32_t z = 0;
+    if (s != 0.0f) {
+        float t = lo / s;
+        float zf = nearbyintf(-128.0f - t);      /* ties to even */
+        z = (int32_t)clampf_range(zf, -128.0f, 127.0f);
+    }
+    for (int64_t k = 0; k < K; ++k) {
+        int32_t qi = 0;
+        if (s != 0.0f) {
+            float rr = nearbyintf(col_vals[k] / s);
+            /* |W / S| stays far below 2^20 (S >= the smallest fp16
+             * subnormal whenever it is non-zero); the bound only keeps the
+             * conversion defined */
+            rr = clampf_range(rr, -1048576.0f, 1048576.0f);
+            qi = (int32_t)rr + z;
+            if (qi > 127) {
+                qi = 127;
+            }
+            if (qi < -128) {
+                qi = -128;
+            }
+        }
+        q_col[k * N] = (int8_t)qi;
+    }
+    *scale_out = s16;
+    *zero_out = (int8_t)z;
+}
+
+/* W fp32 [K,N] -> q int8 [K,N], scales fp16 bits [N], zeros int8 [N]. */
+void oracle_quantize_asym_f32(const float *W, int64_t K, int64_t N, int8_t *q,
+                              uint16_t *scales, int8_t *zeros, float *col_buf)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            col_buf[k] = W[k * N + n];
+        }
+        quantize_column_asym(col_buf, K, q + n, N, &scales[n], &zeros[n]);
+    }
+}
+
+void oracle_quantize_asym_f16(const uint16_t *W, int64_t K, int64_t N, int8_t *q,
+                              uint16_t *scales, int8_t *zeros, float *col_buf)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            col_buf[k] = oracle_f16_to_f32(W[k * N + n]);
+        }
+        quantize_column_asym(col_buf, K, q + n, N, &scales[n], &zeros[n]);
+    }
+}
+
+/* Y[m,n] = S_n * sum_k X[m,k] * (q[k,n] - z_n) + bias_n, in fp64. */
+void oracle_linear_asym(const uint16_t *X, const int8_t *q, const uint16_t *scales,
+                        const int8_t *zeros, const uint16_t *bias, int64_t M,
+                        int64_t K, int64_t N, double *Y, double *acc)
+{
+    for (int64_t row = 0; row < M; ++row) {
+        for (int64_t col = 0; col < N; ++col) {
+            acc[col] = 0.0;
+        }
+        for (int64_t k = 0; k < K; ++k) {
+            double xv = (double)oracle_f16_to_f32(X[row * K + k]);
+            const int8_t *codes = q + k * N;
+            for (int64_t col = 0; col < N; ++col) {
+                acc[col] += xv * (double)((int32_t)codes[col] - (int32_t)zeros[col]);
+            }
+        }
+        for (int64_t col = 0; col < N; ++col) {
+            double out = acc[col] * (double)oracle_f16_to_f32(scales[col]);
+            if (bias) {
+                out += (double)oracle_f16_to_f32(bias[col]);
+            }
+            Y[row * N + col] = out;
+        }
+    }
+}
+
 /* Element-wise array forms of the two conversions (used by the pins). */
 void oracle_f32_to_f16_array(const float *src, int64_t n, uint16_t *dst)
 {

@@ -39,6 +39,17 @@ MUTANTS = {
     "x_row_ignored": ("oracle_f16_to_f32(X[m * K + k])", "oracle_f16_to_f32(X[k])"),
     "scale_indexed_by_row": ("(double)oracle_f16_to_f32(scales[n]);",
                              "(double)oracle_f16_to_f32(scales[m]);"),
+    # asymmetric quantization
+    "asym_256_levels": ("range / 255.0f", "range / 256.0f"),
+    "asym_zero_point_sign": ("nearbyintf(-128.0f - t)", "nearbyintf(-128.0f + t)"),
+    "asym_range_without_zero": ("float lo = 0.0f, hi = 0.0f;", "float lo = col_vals[0], hi = col_vals[0];"),
+    "asym_zero_point_not_added": ("qi = (int32_t)rr + z;", "qi = (int32_t)rr;"),
+    "asym_clip_at_minus_127": ("if (qi < -128) {\n                qi = -128;", "if (qi < -127) {\n                qi = -127;"),
+    "asym_linear_zero_point_dropped": ("(double)((int32_t)codes[col] - (int32_t)zeros[col])", "(double)codes[col]"),
+    "asym_linear_zero_point_added": ("(double)((int32_t)codes[col] - (int32_t)zeros[col])",
+                                     "(double)((int32_t)codes[col] + (int32_t)zeros[col])"),
+    "asym_linear_scale_by_row": ("acc[col] * (double)oracle_f16_to_f32(scales[col])",
+                                 "acc[col] * (double)oracle_f16_to_f32(scales[row])"),
 }
 
 

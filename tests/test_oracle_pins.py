@@ -305,6 +305,103 @@ def pin_tolerance_helper_rejects_a_planted_error(orc):
     assert not oracle.tolerance_ok(orc.linear(X, q, s_bad), Y)[0]
 
 
+# ---------------------------------------------------------------- asymmetric (affine) quantization
+# (q - z) S with S = (hi - lo) / 255 over a range that includes 0 and
+# z = rne(-128 - lo / S): pinned to values fixed by construction.
+
+def pin_asym_integer_grid_round_trips(orc):
+    # W = (i - z) S exactly, with i spanning -128..127 in every column: the
+    # range is exactly 255 S, so the scale, the zero point and every code
+    # come back unchanged
+    rng = np.random.default_rng(41)
+    K, N = 300, 24
+    S = np.array([2.0 ** -e * (1 + f / 1024) for e, f in zip(rng.integers(3, 12, N), rng.integers(0, 1024, N))],
+                 dtype=np.float16)
+    Z = rng.integers(-128, 128, N).astype(np.int32)
+    I = rng.integers(-128, 128, size=(K, N)).astype(np.int32)
+    I[0] = -128
+    I[1] = 127
+    W = ((I - Z) * S.astype(np.float64)).astype(np.float32)
+    assert np.array_equal(W.astype(np.float64), (I - Z) * S.astype(np.float64))   # exact in fp32
+    q, s, z = orc.quantize_asym(W)
+    assert np.array_equal(s.view(np.uint16), S.view(np.uint16))
+    assert np.array_equal(z.astype(np.int32), Z)
+    assert np.array_equal(q.astype(np.int32), I)
+
+
+def pin_asym_zero_weight_is_exact_and_sign_ranges(orc):
+    rng = np.random.default_rng(42)
+    K = 257
+    pos = np.abs(rng.standard_normal(K)).astype(np.float32)
+    neg = -np.abs(rng.standard_normal(K)).astype(np.float32)
+    mixed = rng.standard_normal(K).astype(np.float32)
+    W = np.stack([pos, neg, mixed], axis=1)
+    W[5] = 0.0
+    q, s, z = orc.quantize_asym(W)
+    # 0 is always representable: a zero weight is stored as the zero point
+    assert np.array_equal(q[5], z)
+    # all weights >= 0: the range starts at 0, z = -128, the largest is 127
+    assert z[0] == -128 and q[np.argmax(pos), 0] == 127 and q[:, 0].min() >= -128
+    # all weights <= 0: the range ends at 0, z = 127, the smallest is -128
+    assert z[1] == 127 and q[np.argmin(neg), 1] == -128
+    # mixed signs: the extremes map to the ends of the code range
+    assert q[np.argmin(mixed), 2] == -128 and q[np.argmax(mixed), 2] == 127
+    # strictly positive weights far from 0: the range still starts at 0, so
+    # the smallest weight is NOT on the bottom level
+    lifted = (np.abs(rng.standard_normal((K, 2))) + 1.0).astype(np.float32)
+    ql, sl, zl = orc.quantize_asym(lifted)
+    assert np.all(zl == -128)
+    # with lo = 0 the scale is the symmetric bound's formula over 255 levels
+    top = lifted.max(axis=0)
+    assert np.array_equal(sl, (top / np.float32(255.0)).astype(np.float16))
+    assert np.all(ql.min(axis=0) > -128 + 50)
+    # an all-zero column: scale 0, zero point 0, codes 0
+    q0, s0, z0 = orc.quantize_asym(np.zeros((16, 8), dtype=np.float32))
+    assert not q0.any() and not s0.view(np.uint16).any() and not z0.any()
+
+
+def pin_asym_reconstruction_error_bound(orc):
+    # |w - (q - z) S| <= S / 2, widened by the scale's fp16 rounding, which
+    # can stretch the top of the range by up to 255 * 2^-11 of a level
+    K, N = 512, 96
+    W = synthetic.weights(K, N, SEED, 131, outlier_frac=0.01)
+    W[:, :8] = np.abs(W[:, :8])
+    for Wt in (W, W.astype(np.float16)):
+        q, s, z = orc.quantize_asym(Wt)
+        sf = s.astype(np.float64)
+        deq = (q.astype(np.float64) - z.astype(np.float64)) * sf
+        err = np.abs(deq - Wt.astype(np.float64))
+        assert np.all(err <= (0.5 + 255 * 2.0 ** -11 + 2.0 ** -10) * sf + 1e-12)
+        # the column extremes land within one level of the ends of the code
+        # range (the rounding of S and of z may each move them by a fraction)
+        assert np.all(q.min(axis=0) <= -127) and np.all(q.max(axis=0) >= 126)
+
+
+def pin_asym_linear_unit_rows_and_reductions(orc):
+    rng = np.random.default_rng(43)
+    K, N = 64, 40
+    q = rng.integers(-128, 128, size=(K, N)).astype(np.int8)
+    s = (rng.uniform(0.5, 2.0, N) / 64).astype(np.float16)
+    z = rng.integers(-128, 128, N).astype(np.int8)
+    b = (rng.integers(-64, 64, N) / 8).astype(np.float16)
+    # unit rows pick one dequantized weight row: (q[k] - z) S + bias, exactly
+    ks = [0, 17, 63]
+    X = np.zeros((len(ks), K), dtype=np.float16)
+    X[np.arange(len(ks)), ks] = 1.0
+    Y = orc.linear_asym(X, q, s, z, b)
+    want = (q[ks].astype(np.float64) - z.astype(np.float64)) * s.astype(np.float64) + b.astype(np.float64)
+    assert np.array_equal(Y, want)
+    # a zero point of 0 is the symmetric product
+    Xr = synthetic.activations(5, K, SEED, 132)
+    assert np.array_equal(orc.linear_asym(Xr, q, s, np.zeros(N, np.int8), b), orc.linear(Xr, q, s, b))
+    # shifting every code and its zero point by the same amount changes nothing
+    q2 = np.clip(q.astype(np.int32), -120, 120)
+    z2 = np.clip(z.astype(np.int32), -120, 120)
+    Y1 = orc.linear_asym(Xr, q2.astype(np.int8), s, z2.astype(np.int8))
+    Y2 = orc.linear_asym(Xr, (q2 + 7).astype(np.int8), s, (z2 + 7).astype(np.int8))
+    assert np.allclose(Y1, Y2, rtol=1e-12, atol=1e-12)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
