@@ -91,6 +91,26 @@ int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N,
                             int8_t *q, uint16_t *scales, void *stream);
 
 /*
+ * w8_quantize_per_channel_asym -- per-output-channel ASYMMETRIC (affine)
+ * int8 quantization: the variant the LightSeq 2020 slides compare with the
+ * symmetric one (slide "quantization: clipping + symmetric", where a value
+ * is (i - z) S), with the range, scale and zero point of the
+ * integer-arithmetic quantization paper those slides cite (arXiv
+ * 1712.05877, section 2).  For each channel n:
+ *   lo = min(0, min_k W[k,n]),  hi = max(0, max_k W[k,n])
+ *   S_n = fp16_rne( fp32(hi - lo) / 255 )
+ *   z_n = clamp( rne( -128 - lo / S_n ), -128, 127 )
+ *   q[k,n] = clamp( rne( W[k,n] / S_n ) + z_n, -128, 127 )
+ * (IEEE fp32 operations, S_n widened from fp16; S_n = 0 gives z_n = 0 and
+ * q = 0).  A weight is dequantized as (q - z_n) S_n; 0 is exact.
+ *   zeros   [N] int8 output zero points.
+ * Other arguments, exactness and errors as w8_quantize_per_channel (zeros
+ * must not overlap W, q or scales).
+ */
+int w8_quantize_per_channel_asym(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
+                                 uint16_t *scales, int8_t *zeros, void *stream);
+
+/*
  * w8_prepacked_bytes -- size of the packed weight for a [K, N] q:
  * ceil(N/128) * ceil(K/64) * 8192 bytes (== K*N when K % 64 == 0 and
  * N % 128 == 0).  Returns 0 for K < 1 or N < 1.
@@ -171,6 +191,20 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
 int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
                  const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * w8a16_linear_asym -- Y = X . ((q - z) o S) (+ bias) for codes from
+ * w8_quantize_per_channel_asym: Y[m,n] = S_n sum_k X[m,k] (q[k,n] - z_n)
+ * + bias_n, the expansion of the slides' (i - z) S product with the
+ * activation kept in fp16.  The kernels widen each code to q - z_n, exact
+ * in fp16 (|q - z| <= 255), so the arithmetic and the accuracy bound are
+ * those of w8a16_linear.
+ *   zeros   [N] int8 zero points (must not overlap Y).
+ * Every other argument, the workspace and the errors as w8a16_linear.
+ */
+int w8a16_linear_asym(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
+                      const int8_t *zeros, const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K,
+                      int64_t N, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * w8a16_linear_decode_static -- the decode path of w8a16_linear (M <= 16)

@@ -18,8 +18,8 @@ import os
 import threading
 
 __all__ = [
-    "W8Error", "load_library", "library_path", "quantize", "prepack", "unpack",
-    "prepacked_bytes", "workspace_bytes", "linear", "linear_decode_static", "W8A16Linear", "device_status",
+    "W8Error", "load_library", "library_path", "quantize", "quantize_asym", "prepack", "unpack",
+    "prepacked_bytes", "workspace_bytes", "linear", "linear_asym", "linear_decode_static", "W8A16Linear", "device_status",
     "test_bounded_wait", "STATUS",
 ]
 
@@ -61,6 +61,8 @@ def load_library():
         lib = ctypes.CDLL(_LIB_PATH)
         vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
         lib.w8_quantize_per_channel.argtypes = [vp, i32, i64, i64, vp, vp, vp]
+        lib.w8_quantize_per_channel_asym.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
+        lib.w8a16_linear_asym.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp]
         lib.w8_prepacked_bytes.argtypes = [i64, i64]
         lib.w8_prepacked_bytes.restype = sz
         lib.w8_prepack.argtypes = [vp, i64, i64, vp, vp]
@@ -139,6 +141,36 @@ def quantize(W, q=None, scales=None):
     return q, scales
 
 
+def quantize_asym(W, q=None, scales=None, zeros=None):
+    """Per-output-channel asymmetric (affine) int8 quantization of W [K, N].
+
+    Returns (q int8 [K, N], scales fp16 [N], zeros int8 [N]) on W's device;
+    a weight is dequantized as (q - zero) * scale.
+    """
+    torch = _torch()
+    lib = load_library()
+    _need_cuda(W, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be [K, N]")
+    if W.dtype == torch.float32:
+        dt = W8_F32
+    elif W.dtype == torch.float16:
+        dt = W8_F16
+    else:
+        raise ValueError("W must be float32 or float16")
+    K, N = W.shape
+    if q is None:
+        q = torch.empty((K, N), dtype=torch.int8, device=W.device)
+    if scales is None:
+        scales = torch.empty((N,), dtype=torch.float16, device=W.device)
+    if zeros is None:
+        zeros = torch.empty((N,), dtype=torch.int8, device=W.device)
+    with torch.cuda.device(W.device):
+        _check(lib.w8_quantize_per_channel_asym(_ptr(W), dt, K, N, _ptr(q), _ptr(scales), _ptr(zeros),
+                                                _stream(W.device)), "w8_quantize_per_channel_asym")
+    return q, scales, zeros
+
+
 def prepack(q, out=None):
     """Reorder q [K, N] int8 into the tiled layout (uint8, flat)."""
     torch = _torch()
@@ -204,6 +236,29 @@ def linear(X, packed, scales, bias=None, out=None, workspace=None):
         ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
         _check(lib.w8a16_linear(_ptr(X), _ptr(packed), _ptr(scales), _ptr(bias), _ptr(out),
                                 M, K, N, _ptr(ws), ws_bytes, _stream(X.device)), "w8a16_linear")
+    return out
+
+
+def linear_asym(X, packed, scales, zeros, bias=None, out=None, workspace=None):
+    """Y [M, N] fp16 = X [M, K] fp16 . ((q - zeros) o scales) (+ bias), for
+    codes from quantize_asym."""
+    torch = _torch()
+    lib = load_library()
+    _need_cuda(X, "X")
+    if X.dim() != 2 or X.dtype != torch.float16:
+        raise ValueError("X must be [M, K] float16")
+    M, K = X.shape
+    N = scales.shape[0]
+    if zeros.dtype != torch.int8 or zeros.shape != (N,):
+        raise ValueError("zeros must be [N] int8")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    with torch.cuda.device(X.device):
+        need = int(lib.w8a16_workspace_bytes(M, K, N))
+        ws = workspace if workspace is not None else _workspace(X.device, need)
+        ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+        _check(lib.w8a16_linear_asym(_ptr(X), _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(bias), _ptr(out),
+                                     M, K, N, _ptr(ws), ws_bytes, _stream(X.device)), "w8a16_linear_asym")
     return out
 
 

@@ -433,6 +433,19 @@ __device__ __forceinline__ uint32_t unbias2(uint32_t h2) {
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h2), "r"(0x64806480u));
     return r;
 }
+// With a zero point z (asymmetric codes): the pair minus (1152 + z), i.e.
+// the codes q - z, exact (|q - z| <= 255).  c = zp_bias2(z).
+__device__ __forceinline__ uint32_t unbias2_by(uint32_t h2, uint32_t c) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h2), "r"(c));
+    return r;
+}
+// fp16 1152 + z in both halves: for z in [-128, 127] the value lies in
+// [1024, 1279], where the fp16 pattern is 0x6400 plus (value - 1024).
+__device__ __forceinline__ uint32_t zp_bias2(int z) {
+    const uint32_t h = 0x6480u + (uint32_t)z;
+    return h | (h << 16);
+}
 
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {

@@ -71,6 +71,7 @@ constexpr int kPartialFloats16 = Cfg<2>::kPartialFloats;
 struct Params {
     const uint8_t *packed;
     const uint16_t *scales;
+    const int8_t *zeros;    // zero points (asymmetric codes), else unused
     const uint16_t *bias;   // may be null
     uint16_t *Y;
     int *counters;
@@ -143,7 +144,9 @@ __device__ __forceinline__ void fold(const float (&acc)[MT][NS][4], float (&out)
         }
 }
 
-template <int MT>
+// kZp: asymmetric codes -- every weight is widened to q - z_n (exact in
+// fp16) instead of q; nothing else changes.
+template <int MT, bool kZp>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     using C = Cfg<MT>;
@@ -267,10 +270,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     uint32_t kb = t_begin - first_b * KB;       // its K block
     bool seg_whole = (kb == 0);                 // segment started at K block 0
     bool seg_new = true;
+    // asymmetric codes: 1152 + z of this thread's two channels (rows g, g+8)
+    uint32_t zc_lo = 0x64806480u, zc_hi = 0x64806480u;
 
     for (uint32_t t = t_begin; t < t_end;) {
         if (seg_new) {
             seg_new = false;
+            if constexpr (kZp) {
+                const int64_t n_lo = (int64_t)b * 128 + row_lo;
+                zc_lo = zp_bias2(n_lo < p.N ? p.zeros[n_lo] : 0);
+                zc_hi = zp_bias2(n_lo + 8 < p.N ? p.zeros[n_lo + 8] : 0);
+            }
             if (tail_pair && b == last_b) {
                 if (threadIdx.x == 0) last_flag[0] = (ld_acquire_gpu(&p.counters[b]) == 1);
                 if (!consumers_sync()) return;
@@ -307,10 +317,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                 const uint32_t wh[4] = {ahi.x, ahi.y, ahi.z, ahi.w};
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const uint32_t a0 = unbias2(widen_lo2(wl[jj]));   // row g,   k +0,+1
-                    const uint32_t a1 = unbias2(widen_lo2(wh[jj]));   // row g+8, k +0,+1
-                    const uint32_t a2 = unbias2(widen_hi2(wl[jj]));   // row g,   k +2,+3
-                    const uint32_t a3 = unbias2(widen_hi2(wh[jj]));   // row g+8, k +2,+3
+                    uint32_t a0, a1, a2, a3;
+                    if constexpr (kZp) {
+                        a0 = unbias2_by(widen_lo2(wl[jj]), zc_lo);
+                        a1 = unbias2_by(widen_lo2(wh[jj]), zc_hi);
+                        a2 = unbias2_by(widen_hi2(wl[jj]), zc_lo);
+                        a3 = unbias2_by(widen_hi2(wh[jj]), zc_hi);
+                    } else {
+                        a0 = unbias2(widen_lo2(wl[jj]));   // row g,   k +0,+1
+                        a1 = unbias2(widen_lo2(wh[jj]));   // row g+8, k +0,+1
+                        a2 = unbias2(widen_hi2(wl[jj]));   // row g,   k +2,+3
+                        a3 = unbias2(widen_hi2(wh[jj]));   // row g+8, k +2,+3
+                    }
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
                         const uint4 &xq = xv[mt][jj >> 1];

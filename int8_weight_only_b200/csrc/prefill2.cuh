@@ -84,6 +84,7 @@ constexpr int kPartFloats = kBT * kBNc;
 struct Params {
     const uint8_t *packed;
     const uint16_t *scales;
+    const int8_t *zeros;    // zero points (asymmetric codes), else unused
     const uint16_t *bias;   // may be null
     uint16_t *Y;
     float *partials;        // [pairs][2 slots][2 CTAs][kPartFloats]
@@ -268,7 +269,9 @@ __device__ __forceinline__ void stream_k_share(float *partials, int *counters, u
 // grid = 2 x pairs CTAs, cluster dims (2, 1, 1), kThreads threads,
 // kSmemBytes dynamic shared memory.  tmap_x: X [M, K] fp16, box {64, 128},
 // 128-byte swizzle.
-template <bool kSplit>
+// kZp: asymmetric codes -- the converters widen every weight to q - z_n
+// (exact in fp16) instead of q; nothing else changes.
+template <bool kSplit, bool kZp>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -432,6 +435,11 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         Seg sg;
         while (ok && sched.next(sg)) {
             const bool valid = (sg.tile / p.TT) * 2 + rank < p.NB;
+            uint32_t zc = 0x64806480u;   // 1152 + z of this thread's channel
+            if constexpr (kZp) {
+                const int64_t n = ((int64_t)(sg.tile / p.TT) * 2 + rank) * kBNc + r;
+                if (valid && n < p.N) zc = zp_bias2(p.zeros[n]);
+            }
             for (int ks = sg.ks0; ks < sg.ks1; ++ks) {
                 const int cnt = min(kKStep, p.KB - kKStep * ks);
                 if (!warp_all(mbar_wait(&w_full[wr.s], wr.ph, SITE_P2_WFULL))) { ok = false; break; }
@@ -460,8 +468,13 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                         const uint32_t w[4] = {c[t][i].x, c[t][i].y, c[t][i].z, c[t][i].w};
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            v[8 * i + 2 * j] = unbias2(widen_lo2(w[j]));
-                            v[8 * i + 2 * j + 1] = unbias2(widen_hi2(w[j]));
+                            if constexpr (kZp) {
+                                v[8 * i + 2 * j] = unbias2_by(widen_lo2(w[j]), zc);
+                                v[8 * i + 2 * j + 1] = unbias2_by(widen_hi2(w[j]), zc);
+                            } else {
+                                v[8 * i + 2 * j] = unbias2(widen_lo2(w[j]));
+                                v[8 * i + 2 * j + 1] = unbias2(widen_hi2(w[j]));
+                            }
                         }
                     }
                     tmem_st_32x32b_x32(lane_addr + kAcol0 + 32 * kKStep * ar.s + 32 * t, v);

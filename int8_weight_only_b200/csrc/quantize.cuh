@@ -88,6 +88,35 @@ __device__ __forceinline__ int quantize_exact(float w, float s) {
     return max(-127, min(127, v));
 }
 
+// The asymmetric form: clamp(rne(w / s) + z, -128, 127).  There |w / s|
+// stays below about 255.2 (|w| is at most the range hi - lo, and s is that
+// range over 255 up to the fp16 rounding of s), so the same argument holds
+// with 256 in place of 126: r and fl(w/s) are within 2^-15 + 2^-16 of each
+// other, and r more than 2^-13 from every half-integer decides the code.
+__device__ __forceinline__ int quantize_fast_asym(float w, float inv_s, int z, bool &sure) {
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+    const float r = w * inv_s;
+    const float t = r + kMagic;
+    const float d = fabsf(r - (t - kMagic));
+    sure = (fabsf(r) < 256.0f) & (d < 0.5f - 0x1p-13f);
+    return max(-128, min(127, (__float_as_int(t) - 0x4B400000) + z));
+}
+__device__ __forceinline__ int quantize_exact_asym(float w, float s, int z) {
+    if (s == 0.0f) return 0;
+    // |w / s| < 2^20 whenever s is non-zero (s >= the smallest fp16 subnormal)
+    const float r = fminf(fmaxf(__fdiv_rn(w, s), -1048576.0f), 1048576.0f);
+    return max(-128, min(127, __float2int_rn(r) + z));
+}
+
+// Scale and zero point of a channel from its range [lo, hi] (lo <= 0 <= hi):
+// s = fp16_rne(fp32(hi - lo) / 255), z = clamp(rne(-128 - lo / s), -128, 127).
+__device__ __forceinline__ void asym_params(float lo, float hi, __half &s16, int &z) {
+    s16 = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 255.0f));
+    const float s = __half2float(s16);
+    z = 0;
+    if (s != 0.0f) z = max(-128, min(127, __float2int_rn(__fsub_rn(-128.0f, __fdiv_rn(lo, s)))));
+}
+
 // The 16-byte row segment of a thread, widened to fp32.
 template <typename T>
 __device__ __forceinline__ void load_seg(const uint8_t *p, float (&v)[Box<T>::kCols]);
@@ -111,6 +140,7 @@ __device__ __forceinline__ void load_seg<__half>(const uint8_t *p, float (&v)[8]
 struct Params {
     int8_t *q;
     uint16_t *scales;
+    int8_t *zeros;     // asymmetric form only: [N] zero points
     int64_t K;
     int64_t N;
     int kc;            // rows per cluster rank (multiple of the box height)
@@ -133,7 +163,11 @@ struct Params {
 // which waited for the peers' (c) of step j-1, issued after their reads of
 // P_{j-2} -- the values part[j % 3] held before -- so three buffers never
 // race.  The exchange barriers alternate by panel parity.
-template <typename T>
+//
+// kAsym: the asymmetric form -- pass 1 keeps the column minimum and maximum
+// (both start at 0: the range always holds 0), the exchange combines both,
+// and pass 2 writes clamp(rne(w / s) + z, -128, 127).
+template <typename T, bool kAsym>
 __global__ void __launch_bounds__(kThreads, 2)
 quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
     using B = Box<T>;
@@ -147,6 +181,10 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
     __shared__ float red[kConsumerWarps][kPanel];
     __shared__ float col_scale[kPanel];
     __shared__ float col_inv[kPanel];
+    // asymmetric form: partial minima, and the zero points
+    __shared__ float part_lo[kAsym ? kPartBufs : 1][kPanel];
+    __shared__ float red_lo[kAsym ? kConsumerWarps : 1][kPanel];
+    __shared__ int col_zero[kPanel];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -224,9 +262,9 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
         for (int j = 0; j <= npan && ok; ++j) {
             // ---------------- (a) pass 1 over panel j: column |max|
             if (j < npan) {
-                float amax[B::kCols];
+                float amax[B::kCols], amin[B::kCols];   // amin: asymmetric form only
 #pragma unroll
-                for (int e = 0; e < B::kCols; ++e) amax[e] = 0.0f;
+                for (int e = 0; e < B::kCols; ++e) amax[e] = amin[e] = 0.0f;
                 for (int i = 0; i < nbox; ++i) {
                     if (!warp_all(mbar_wait_parked(&full[s], ph, SITE_Q_LOAD))) { ok = false; break; }
                     const uint8_t *box = ring + s * kBoxBytes;
@@ -234,8 +272,16 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                     for (int w = 0; w < B::kSweeps; ++w) {
                         float v[B::kCols];
                         load_seg<T>(box + (rsub + w * B::kSweep) * B::kRowBytes + 16 * t, v);
+                        if constexpr (kAsym) {
 #pragma unroll
-                        for (int e = 0; e < B::kCols; ++e) amax[e] = fmaxf(amax[e], fabsf(v[e]));
+                            for (int e = 0; e < B::kCols; ++e) {
+                                amax[e] = fmaxf(amax[e], v[e]);
+                                amin[e] = fminf(amin[e], v[e]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < B::kCols; ++e) amax[e] = fmaxf(amax[e], fabsf(v[e]));
+                        }
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
@@ -246,11 +292,16 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
 #pragma unroll
                 for (int off = B::kThreadsPerRow; off < 32; off <<= 1)
 #pragma unroll
-                    for (int e = 0; e < B::kCols; ++e)
+                    for (int e = 0; e < B::kCols; ++e) {
                         amax[e] = fmaxf(amax[e], __shfl_xor_sync(0xffffffffu, amax[e], off));
+                        if constexpr (kAsym) amin[e] = fminf(amin[e], __shfl_xor_sync(0xffffffffu, amin[e], off));
+                    }
                 if (lane < B::kThreadsPerRow) {
 #pragma unroll
-                    for (int e = 0; e < B::kCols; ++e) red[warp][col0 + e] = amax[e];
+                    for (int e = 0; e < B::kCols; ++e) {
+                        red[warp][col0 + e] = amax[e];
+                        if constexpr (kAsym) red_lo[warp][col0 + e] = amin[e];
+                    }
                 }
                 if (!csync()) { ok = false; break; }
                 if (c < kPanel) {
@@ -258,6 +309,12 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
 #pragma unroll
                     for (int w = 0; w < kConsumerWarps; ++w) m = fmaxf(m, red[w][c]);
                     part[j % kPartBufs][c] = m;
+                    if constexpr (kAsym) {
+                        float lo = 0.0f;
+#pragma unroll
+                        for (int w = 0; w < kConsumerWarps; ++w) lo = fminf(lo, red_lo[w][c]);
+                        part_lo[j % kPartBufs][c] = lo;
+                    }
                 }
             }
             if (j == 0) {
@@ -274,12 +331,25 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                 float m = 0.0f;
                 const uint32_t local = smem_u32(&part[pj % kPartBufs][c]);
                 for (uint32_t r = 0; r < csize; ++r) m = fmaxf(m, ld_dsmem_f32(mapa_shared(local, r)));
-                const __half s16 = __float2half_rn(__fdiv_rn(m, 127.0f));
+                __half s16;
+                int z = 0;
+                if constexpr (kAsym) {
+                    float lo = 0.0f;
+                    const uint32_t local_lo = smem_u32(&part_lo[pj % kPartBufs][c]);
+                    for (uint32_t r = 0; r < csize; ++r) lo = fminf(lo, ld_dsmem_f32(mapa_shared(local_lo, r)));
+                    asym_params(lo, m, s16, z);
+                } else {
+                    s16 = __float2half_rn(__fdiv_rn(m, 127.0f));
+                }
                 const float sf = __half2float(s16);
                 col_scale[c] = sf;
                 col_inv[c] = sf != 0.0f ? __frcp_rn(sf) : 0.0f;
+                col_zero[c] = z;
                 const int64_t n = (int64_t)panel * kPanel + c;
-                if (rank == 0 && n < p.N) p.scales[n] = __half_as_ushort(s16);
+                if (rank == 0 && n < p.N) {
+                    p.scales[n] = __half_as_ushort(s16);
+                    if constexpr (kAsym) p.zeros[n] = (int8_t)z;
+                }
             }
             // every consumer's partial maxima of panel j are in part[] and
             // every read of panel j - 1's values is done
@@ -289,10 +359,12 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                 mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[j & 1]), (uint32_t)c));
             // ---------------- (d) pass 2 over panel j - 1 (from L2)
             float sc[B::kCols], inv[B::kCols];
+            int zp[B::kCols];   // asymmetric form only
 #pragma unroll
             for (int e = 0; e < B::kCols; ++e) {
                 sc[e] = col_scale[col0 + e];
                 inv[e] = col_inv[col0 + e];
+                zp[e] = col_zero[col0 + e];
             }
             const int64_t n0 = (int64_t)panel * kPanel + col0;
             const bool cols_ok = n0 < p.N;   // N % 8 == 0: a segment is all in or all out
@@ -309,12 +381,20 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
 #pragma unroll
                     for (int e = 0; e < B::kCols; ++e) {
                         bool se;
-                        code[e] = quantize_fast(v[e], inv[e], se);
+                        if constexpr (kAsym)
+                            code[e] = quantize_fast_asym(v[e], inv[e], zp[e], se);
+                        else
+                            code[e] = quantize_fast(v[e], inv[e], se);
                         sure &= se;
                     }
                     if (!sure) {   // rare: some product lies near a rounding boundary
 #pragma unroll
-                        for (int e = 0; e < B::kCols; ++e) code[e] = quantize_exact(v[e], sc[e]);
+                        for (int e = 0; e < B::kCols; ++e) {
+                            if constexpr (kAsym)
+                                code[e] = quantize_exact_asym(v[e], sc[e], zp[e]);
+                            else
+                                code[e] = quantize_exact(v[e], sc[e]);
+                        }
                     }
                     uint32_t packed[B::kCols / 4];
 #pragma unroll

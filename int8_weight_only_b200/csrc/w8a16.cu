@@ -30,6 +30,8 @@ struct DeviceInfo {
     // resident quantize clusters per cluster size (0 = not yet queried)
     int qclusters_f32[quant::kMaxCluster + 1] = {};
     int qclusters_f16[quant::kMaxCluster + 1] = {};
+    int qclusters_asym_f32[quant::kMaxCluster + 1] = {};
+    int qclusters_asym_f16[quant::kMaxCluster + 1] = {};
 };
 
 std::mutex g_mu;
@@ -51,34 +53,25 @@ int device_info(DeviceInfo **out) {
         d.status = (major == 10 && minor == 0) ? W8_OK : W8_ERR_DEVICE;
         if (d.status == W8_OK) {
             cudaError_t e = cudaSuccess;
-            e = cudaFuncSetAttribute(decode::decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     decode::Cfg<1>::kSmemBytes);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(decode::decode_kernel<2>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         decode::Cfg<2>::kSmemBytes);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(decode::decode_kernel<4>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         decode::Cfg<4>::kSmemBytes);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(decode::decode_kernel<8>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         decode::Cfg<8>::kSmemBytes);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(prefill2::prefill2_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         prefill2::kSmemBytes);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(prefill2::prefill2_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         prefill2::kSmemBytes);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(quant::quantize_kernel<float>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, quant::kSmemBytes);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(quant::quantize_kernel<__half>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, quant::kSmemBytes);
+            auto smem = [&e](const void *fn, int bytes) {
+                if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+            };
+            smem((const void *)decode::decode_kernel<1, false>, decode::Cfg<1>::kSmemBytes);
+            smem((const void *)decode::decode_kernel<2, false>, decode::Cfg<2>::kSmemBytes);
+            smem((const void *)decode::decode_kernel<4, false>, decode::Cfg<4>::kSmemBytes);
+            smem((const void *)decode::decode_kernel<8, false>, decode::Cfg<8>::kSmemBytes);
+            smem((const void *)decode::decode_kernel<1, true>, decode::Cfg<1>::kSmemBytes);
+            smem((const void *)decode::decode_kernel<2, true>, decode::Cfg<2>::kSmemBytes);
+            smem((const void *)decode::decode_kernel<4, true>, decode::Cfg<4>::kSmemBytes);
+            smem((const void *)decode::decode_kernel<8, true>, decode::Cfg<8>::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<false, false>, prefill2::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<true, false>, prefill2::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<false, true>, prefill2::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<true, true>, prefill2::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<float, false>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<__half, false>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<float, true>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<__half, true>, quant::kSmemBytes);
             if (e != cudaSuccess) return W8_ERR_CUDA;
         }
         d.ready = true;
@@ -139,9 +132,9 @@ inline int quantize_cluster(int64_t K, int rows_per_box) {
     return (int)std::max<int64_t>(1, std::min<int64_t>(4, cdiv(K, 2 * rows_per_box)));
 }
 
-template <typename T>
+template <typename T, bool kAsym>
 int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_t K, int64_t N,
-                    int8_t *q, uint16_t *scales, cudaStream_t st) {
+                    int8_t *q, uint16_t *scales, int8_t *zeros, cudaStream_t st) {
     constexpr int rows = quant::Box<T>::kRows;
     const int C = quantize_cluster(K, rows);
     const int64_t kc = cdiv(cdiv(K, C), rows) * rows;
@@ -168,11 +161,13 @@ int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_
     int resident = 0;
     {
         std::lock_guard<std::mutex> lock(g_mu);
-        int &cached = sizeof(T) == 4 ? d->qclusters_f32[C] : d->qclusters_f16[C];
+        int &cached = kAsym ? (sizeof(T) == 4 ? d->qclusters_asym_f32[C] : d->qclusters_asym_f16[C])
+                            : (sizeof(T) == 4 ? d->qclusters_f32[C] : d->qclusters_f16[C]);
         if (cached == 0) {
             cfg.gridDim = dim3((unsigned)(C * d->sms), 1, 1);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, quant::quantize_kernel<T>, &cfg) != cudaSuccess || n < 1) {
+            if (cudaOccupancyMaxActiveClusters(&n, quant::quantize_kernel<T, kAsym>, &cfg) != cudaSuccess ||
+                n < 1) {
                 cudaGetLastError();
                 n = std::max(1, d->sms / C);
             }
@@ -183,13 +178,14 @@ int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_
     quant::Params p;
     p.q = q;
     p.scales = scales;
+    p.zeros = zeros;
     p.K = K;
     p.N = N;
     p.kc = (int)kc;
     p.panels = (int)panels;
     p.clusters = (int)std::min<int64_t>(panels, resident);
     cfg.gridDim = dim3((unsigned)(p.clusters * C), 1, 1);
-    if (cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T>, map, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T, kAsym>, map, p) != cudaSuccess) {
         cudaGetLastError();
         return W8_ERR_CUDA;
     }
@@ -198,7 +194,7 @@ int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_
 
 // Programmatic dependent launch: this kernel's prologue and an L2 prefetch
 // of its first weight tiles overlap the previous kernel in the stream.
-template <int MT>
+template <int MT, bool kZp>
 int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G, 1, 1);
@@ -210,7 +206,7 @@ int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode::decode_kernel<MT>, map, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, decode::decode_kernel<MT, kZp>, map, p) != cudaSuccess) {
         cudaGetLastError();
         return W8_ERR_CUDA;
     }
@@ -219,8 +215,8 @@ int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t 
 
 // Tensor-core linear for M > 64 on CTA pairs (prefill2.cuh).
 int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
-                    const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N, float *partials,
-                    int *counters, cudaStream_t st) {
+                    const int8_t *zeros, const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
+                    float *partials, int *counters, cudaStream_t st) {
     CUtensorMap map;
     int rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
                          prefill2::kBTc, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -228,6 +224,7 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
     prefill2::Params p;
     p.packed = packed;
     p.scales = scales;
+    p.zeros = zeros;
     p.bias = bias;
     p.Y = Y;
     p.partials = partials;
@@ -259,7 +256,8 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
         if (d->pairs == 0) {
             cfg.gridDim = dim3((unsigned)d->sms, 1, 1);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, prefill2::prefill2_kernel<false>, &cfg) != cudaSuccess || n < 1) {
+            if (cudaOccupancyMaxActiveClusters(&n, prefill2::prefill2_kernel<false, false>, &cfg) != cudaSuccess ||
+                n < 1) {
                 cudaGetLastError();
                 n = d->sms / 2;
             }
@@ -300,8 +298,13 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
         p.sk_iters = 0;
     }
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-    const cudaError_t e = split ? cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<true>, map, p)
-                                : cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<false>, map, p);
+    cudaError_t e;
+    if (zeros)
+        e = split ? cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<true, true>, map, p)
+                  : cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<false, true>, map, p);
+    else
+        e = split ? cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<true, false>, map, p)
+                  : cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<false, false>, map, p);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return W8_ERR_CUDA;
@@ -334,26 +337,45 @@ const char *w8_error_string(int status) {
     }
 }
 
-int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
-                            uint16_t *scales, void *stream) {
+// Both quantization forms: zeros == nullptr selects the symmetric one.
+static int quantize_common(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q, uint16_t *scales,
+                           int8_t *zeros, bool asym, void *stream) {
     if (w_dtype != W8_F32 && w_dtype != W8_F16) return W8_ERR_DTYPE;
     if (K < 1 || N < 0 || N % 8 != 0 || K > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX * 8)
         return W8_ERR_SHAPE;
     if (N == 0) return W8_OK;   // nothing to read or write: pointers may be NULL
-    if (!W || !q || !scales) return W8_ERR_NULL;
+    if (!W || !q || !scales || (asym && !zeros)) return W8_ERR_NULL;
     if (!aligned16(W) || !aligned16(q) || !aligned16(scales)) return W8_ERR_ALIGN;
     const size_t welem = w_dtype == W8_F32 ? 4 : 2;
     if (overlap(W, (size_t)K * N * welem, q, (size_t)K * N) ||
         overlap(W, (size_t)K * N * welem, scales, (size_t)N * 2) ||
         overlap(q, (size_t)K * N, scales, (size_t)N * 2))
         return W8_ERR_ALIAS;
+    if (asym && (overlap(zeros, (size_t)N, W, (size_t)K * N * welem) || overlap(zeros, (size_t)N, q, (size_t)K * N) ||
+                 overlap(zeros, (size_t)N, scales, (size_t)N * 2)))
+        return W8_ERR_ALIAS;
     DeviceInfo *d = nullptr;
     int rc = device_info(&d);
     if (rc != W8_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (asym) {
+        if (w_dtype == W8_F32)
+            return launch_quantize<float, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, zeros, st);
+        return launch_quantize<__half, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, zeros, st);
+    }
     if (w_dtype == W8_F32)
-        return launch_quantize<float>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, st);
-    return launch_quantize<__half>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, st);
+        return launch_quantize<float, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, nullptr, st);
+    return launch_quantize<__half, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, nullptr, st);
+}
+
+int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
+                            uint16_t *scales, void *stream) {
+    return quantize_common(W, w_dtype, K, N, q, scales, nullptr, false, stream);
+}
+
+int w8_quantize_per_channel_asym(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
+                                 uint16_t *scales, int8_t *zeros, void *stream) {
+    return quantize_common(W, w_dtype, K, N, q, scales, zeros, true, stream);
 }
 
 size_t w8_prepacked_bytes(int64_t K, int64_t N) {
@@ -427,13 +449,14 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N) {
     return workspace_total(d->sms, N);
 }
 
-int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
-                 const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
-                 void *workspace, size_t workspace_bytes, void *stream) {
+// Both code forms: zeros == nullptr selects the symmetric one.
+static int linear_common(const uint16_t *X, const uint8_t *packed, const uint16_t *scales, const int8_t *zeros,
+                         bool asym, const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
+                         void *workspace, size_t workspace_bytes, void *stream) {
     if (M < 0 || K < 1 || N < 1 || K % 8 != 0 || N % 8 != 0 || M > (int64_t)INT32_MAX ||
         K > (int64_t)INT32_MAX || cdiv(K, 64) > INT32_MAX)
         return W8_ERR_SHAPE;
-    if (!packed || !scales) return W8_ERR_NULL;
+    if (!packed || !scales || (asym && !zeros)) return W8_ERR_NULL;
     if (M == 0) return W8_OK;   // empty batch: X and Y may be NULL
     if (!X || !Y) return W8_ERR_NULL;
     if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(Y) ||
@@ -442,7 +465,8 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
     const size_t ybytes = (size_t)M * N * 2;
     if (overlap(Y, ybytes, X, (size_t)M * K * 2) ||
         overlap(Y, ybytes, packed, w8_prepacked_bytes(K, N)) ||
-        overlap(Y, ybytes, scales, (size_t)N * 2) || (bias && overlap(Y, ybytes, bias, (size_t)N * 2)))
+        overlap(Y, ybytes, scales, (size_t)N * 2) || (bias && overlap(Y, ybytes, bias, (size_t)N * 2)) ||
+        (asym && overlap(Y, ybytes, zeros, (size_t)N)))
         return W8_ERR_ALIAS;
     DeviceInfo *d = nullptr;
     int rc = device_info(&d);
@@ -467,6 +491,7 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
         decode::Params p;
         p.packed = packed;
         p.scales = scales;
+        p.zeros = zeros;
         p.bias = bias;
         p.Y = Y;
         p.partials = partials;
@@ -479,15 +504,37 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
         if ((uint64_t)T * (uint64_t)(G + 1) >= (1ull << 32)) return W8_ERR_SHAPE;
         p.T = (uint32_t)T;
         p.G = (uint32_t)G;
+        if (asym) {
+            switch (MT) {
+                case 1: return launch_decode<1, true>(map, p, st);
+                case 2: return launch_decode<2, true>(map, p, st);
+                case 4: return launch_decode<4, true>(map, p, st);
+                default: return launch_decode<8, true>(map, p, st);
+            }
+        }
         switch (MT) {
-            case 1: return launch_decode<1>(map, p, st);
-            case 2: return launch_decode<2>(map, p, st);
-            case 4: return launch_decode<4>(map, p, st);
-            default: return launch_decode<8>(map, p, st);
+            case 1: return launch_decode<1, false>(map, p, st);
+            case 2: return launch_decode<2, false>(map, p, st);
+            case 4: return launch_decode<4, false>(map, p, st);
+            default: return launch_decode<8, false>(map, p, st);
         }
     }
 
-    return launch_prefill2(d, X, packed, scales, bias, Y, M, K, N, partials, counters, st);
+    return launch_prefill2(d, X, packed, scales, asym ? zeros : nullptr, bias, Y, M, K, N, partials, counters,
+                           st);
+}
+
+int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
+                 const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
+                 void *workspace, size_t workspace_bytes, void *stream) {
+    return linear_common(X, packed, scales, nullptr, false, bias, Y, M, K, N, workspace, workspace_bytes,
+                         stream);
+}
+
+int w8a16_linear_asym(const uint16_t *X, const uint8_t *packed, const uint16_t *scales, const int8_t *zeros,
+                      const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N, void *workspace,
+                      size_t workspace_bytes, void *stream) {
+    return linear_common(X, packed, scales, zeros, true, bias, Y, M, K, N, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- diagnostics
@@ -608,6 +655,7 @@ extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *pack
     decode::Params p;
     p.packed = packed;
     p.scales = scales;
+    p.zeros = nullptr;
     p.bias = bias;
     p.Y = Y;
     p.partials = static_cast<float *>(scratch);
@@ -621,8 +669,8 @@ extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *pack
     p.T = (uint32_t)T;
     p.G = (uint32_t)G;
     if (MT == 1)
-        decode::decode_kernel<1><<<p.G, decode::kThreads, decode::Cfg<1>::kSmemBytes, st>>>(map, p);
+        decode::decode_kernel<1, false><<<p.G, decode::kThreads, decode::Cfg<1>::kSmemBytes, st>>>(map, p);
     else
-        decode::decode_kernel<2><<<p.G, decode::kThreads, decode::Cfg<2>::kSmemBytes, st>>>(map, p);
+        decode::decode_kernel<2, false><<<p.G, decode::kThreads, decode::Cfg<2>::kSmemBytes, st>>>(map, p);
     return launch_status();
 }
