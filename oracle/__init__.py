@@ -63,6 +63,9 @@ class Oracle:
         lib.oracle_quantize_asym_f32.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         lib.oracle_quantize_asym_f16.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         lib.oracle_linear_asym.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
+        lib.oracle_quantize_clip.argtypes = [vp, ctypes.c_int, i64, i64, ctypes.c_int, ctypes.c_double,
+                                             vp, vp, vp, vp]
+        lib.oracle_quantize_clip.restype = None
         for f in ("oracle_f32_to_f16_array", "oracle_f16_to_f32_array",
                   "oracle_quantize_f32", "oracle_quantize_f16", "oracle_linear",
                   "oracle_quantize_asym_f32", "oracle_quantize_asym_f16", "oracle_linear_asym"):
@@ -149,6 +152,31 @@ class Oracle:
             raise TypeError("W must be float32 or float16")
         return q, s.view(np.float16), z
 
+    def quantize_clip(self, W: np.ndarray, mode: str, param: float):
+        """Clipped symmetric int8 quantization (same code format as
+        ``quantize``).  mode "fixed": bound = min(max|W|, param); mode
+        "percentile": bound = the ceil(param K)-th smallest |W| per channel.
+        Returns (q int8 [K, N], scales float16 [N])."""
+        if W.ndim != 2:
+            raise ValueError("W must be 2-D [K, N]")
+        modes = {"fixed": 0, "percentile": 1}
+        if mode not in modes:
+            raise ValueError("mode must be 'fixed' or 'percentile'")
+        K, N = W.shape
+        q = np.empty((K, N), dtype=np.int8)
+        s = np.empty(N, dtype=np.uint16)
+        buf = np.empty(max(K, 1), dtype=np.float32)
+        sbuf = np.empty(max(K, 1), dtype=np.float32)
+        if W.dtype == np.float32:
+            Wc, f16 = np.ascontiguousarray(W), 0
+        elif W.dtype == np.float16:
+            Wc, f16 = np.ascontiguousarray(W).view(np.uint16), 1
+        else:
+            raise TypeError("W must be float32 or float16")
+        self.lib.oracle_quantize_clip(_ptr(Wc), f16, K, N, modes[mode], float(param), _ptr(q), _ptr(s),
+                                      _ptr(buf), _ptr(sbuf))
+        return q, s.view(np.float16)
+
     def linear_asym(self, X, q, scales, zeros, bias=None) -> np.ndarray:
         """Y = X . ((q - zeros) o scales) (+ bias) in fp64 (not rounded)."""
         M, K = X.shape
@@ -197,6 +225,10 @@ def quantize_asym(W):
 
 def linear_asym(X, q, scales, zeros, bias=None):
     return default().linear_asym(X, q, scales, zeros, bias)
+
+
+def quantize_clip(W, mode, param):
+    return default().quantize_clip(W, mode, param)
 
 
 def tolerance_ok(y_test: np.ndarray, y_ref: np.ndarray):

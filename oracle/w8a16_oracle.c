@@ -36,6 +36,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* ---------------------------------------------------------------------
@@ -222,6 +223,87 @@ void oracle_linear(const uint16_t *X, const int8_t *q, const uint16_t *scales,
             }
             Y[m * N + n] = y;
         }
+    }
+}
+
+/* ---------------------------------------------------------------------
+ * Clipped symmetric quantization -- the calibration choices the LightSeq
+ * 2020 slides evaluate ("fixed range clip" and "percentage clip" against
+ * plain max|W|, slide "quantization: clipping + symmetric").  The bound
+ * that is put on level 127 is, per channel n:
+ *   fixed range:  bound_n = min( max_k |W[k,n]|, c )        (c >= 0)
+ *   percentage:   bound_n = the r-th smallest |W[k,n]|,
+ *                 r = clamp( ceil(p K), 1, K ) in IEEE double  (0 < p <= 1)
+ * and then, as in the symmetric quantizer, S = fp16_rne(fp32(bound)/127)
+ * and q = clamp(rne(W / S), -127, 127): weights beyond the bound land on
+ * +-127.  c = +inf and p = 1 are the plain symmetric quantizer.
+ * ------------------------------------------------------------------- */
+
+static float clampf_range(float v, float lo, float hi);
+
+static int compare_floats(const void *a, const void *b)
+{
+    float x = *(const float *)a, y = *(const float *)b;
+    return (x > y) - (x < y);
+}
+
+/* The codes of one column for a given bound (the symmetric quantizer's
+ * second half). */
+static void codes_for_bound(const float *col_vals, int64_t K, float bound, int8_t *q_col,
+                            int64_t N, uint16_t *scale_out)
+{
+    uint16_t s16 = oracle_f32_to_f16(bound / 127.0f);
+    float s = oracle_f16_to_f32(s16);
+    for (int64_t k = 0; k < K; ++k) {
+        int32_t qi = 0;
+        if (s != 0.0f) {
+            float rr = nearbyintf(col_vals[k] / s);
+            rr = clampf_range(rr, -127.0f, 127.0f);
+            qi = (int32_t)rr;
+        }
+        q_col[k * N] = (int8_t)qi;
+    }
+    *scale_out = s16;
+}
+
+/* mode 0: fixed range (param = c); mode 1: percentage (param = p).
+ * col_buf: K floats; sort_buf: K floats. */
+static void quantize_clip_column(const float *col_vals, int64_t K, int mode, double param,
+                                 int8_t *q_col, int64_t N, uint16_t *scale_out, float *sort_buf)
+{
+    float bound = 0.0f;
+    if (mode == 0) {
+        for (int64_t k = 0; k < K; ++k) {
+            float mag = fabsf(col_vals[k]);
+            if (mag > bound) {
+                bound = mag;
+            }
+        }
+        if ((double)bound > param) {
+            bound = (float)param;
+        }
+    } else {
+        double rr = ceil(param * (double)K);
+        int64_t r = rr < 1.0 ? 1 : (rr > (double)K ? K : (int64_t)rr);
+        for (int64_t k = 0; k < K; ++k) {
+            sort_buf[k] = fabsf(col_vals[k]);
+        }
+        qsort(sort_buf, (size_t)K, sizeof(float), compare_floats);
+        bound = sort_buf[r - 1];
+    }
+    codes_for_bound(col_vals, K, bound, q_col, N, scale_out);
+}
+
+/* W fp32 [K,N] or fp16 bits [K,N] (w_is_f16) -> q int8 [K,N], scales. */
+void oracle_quantize_clip(const void *W, int w_is_f16, int64_t K, int64_t N, int mode, double param,
+                          int8_t *q, uint16_t *scales, float *col_buf, float *sort_buf)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            col_buf[k] = w_is_f16 ? oracle_f16_to_f32(((const uint16_t *)W)[k * N + n])
+                                  : ((const float *)W)[k * N + n];
+        }
+        quantize_clip_column(col_buf, K, mode, param, q + n, N, &scales[n], sort_buf);
     }
 }
 

@@ -402,6 +402,66 @@ def pin_asym_linear_unit_rows_and_reductions(orc):
     assert np.allclose(Y1, Y2, rtol=1e-12, atol=1e-12)
 
 
+# ---------------------------------------------------------------- clipped scale
+# bound = min(max|W|, c) or the ceil(pK)-th smallest |W| per channel, then
+# the symmetric quantizer: pinned to order statistics known by construction.
+
+def pin_clip_reduces_to_symmetric(orc):
+    W = synthetic.weights(300, 48, SEED, 141, outlier_frac=0.01)
+    q, s = orc.quantize(W)
+    for mode, param in (("percentile", 1.0), ("fixed", float("inf")), ("fixed", 1e30)):
+        qc, sc = orc.quantize_clip(W, mode, param)
+        assert np.array_equal(qc, q) and np.array_equal(sc.view(np.uint16), s.view(np.uint16))
+
+
+def pin_percentile_bound_is_the_order_statistic(orc):
+    # each column holds |w| = delta, 2 delta, ..., K delta (shuffled, random
+    # signs): the r-th smallest magnitude is r delta exactly
+    rng = np.random.default_rng(44)
+    K, N, delta = 400, 12, 2.0 ** -10
+    W = np.empty((K, N), dtype=np.float32)
+    for n in range(N):
+        W[:, n] = rng.permutation(np.arange(1, K + 1)) * delta * rng.choice([-1.0, 1.0], K)
+    for p, r in ((0.9501, 381), (0.5, 200), (0.999, 400), (0.0001, 1), (0.75, 300)):
+        q, s = orc.quantize_clip(W, "percentile", p)
+        want = np.float16(np.float32(r * delta) / np.float32(127.0))
+        assert np.all(s == want), (p, r)
+        # everything at or beyond the bound is clipped onto +-127, nothing
+        # well below it is
+        mag = np.abs(W)
+        assert np.all(np.abs(q[mag >= r * delta]) == 127), (p, r)
+        assert np.all(np.abs(q[mag < 0.99 * r * delta]) < 127), (p, r)
+
+
+def pin_percentile_monotone_in_p(orc):
+    W = synthetic.weights(512, 40, SEED, 142, outlier_frac=0.01)
+    prev = None
+    for p in (0.5, 0.9, 0.99, 0.999, 1.0):
+        _, s = orc.quantize_clip(W, "percentile", p)
+        sf = s.astype(np.float64)
+        if prev is not None:
+            assert np.all(sf >= prev)
+        prev = sf
+
+
+def pin_fixed_clip_scale_and_codes(orc):
+    W = synthetic.weights(256, 32, SEED, 143, outlier_frac=0.01)
+    c = 127.0 * 2.0 ** -12         # below every column's max: S = 2^-12 exactly
+    assert np.all(np.abs(W).max(axis=0) > c)
+    q, s = orc.quantize_clip(W, "fixed", c)
+    assert np.all(s == np.float16(2.0 ** -12))
+    inside = np.abs(W) <= c
+    err = np.abs(q.astype(np.float64) * 2.0 ** -12 - W.astype(np.float64))
+    assert np.all(err[inside] <= 2.0 ** -13)
+    assert np.all(np.abs(q[np.abs(W) >= c * (1 + 2 ** -7)]) == 127)
+    # a clip above a column's max leaves that column unclipped
+    W2 = W.copy()
+    W2[:, 5] *= 0.1
+    q2, s2 = orc.quantize_clip(W2, "fixed", c)
+    qs, ss = orc.quantize(W2[:, 5:6])
+    assert s2[5] == ss[0] and np.array_equal(q2[:, 5], qs[:, 0])
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
