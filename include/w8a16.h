@@ -111,6 +111,29 @@ int w8_quantize_per_channel_asym(const void *W, int w_dtype, int64_t K, int64_t 
                                  uint16_t *scales, int8_t *zeros, void *stream);
 
 /*
+ * w8_quantize_per_channel_clip -- symmetric int8 quantization with a
+ * clipped bound: the "fixed range clip" and "percentage clip" calibrations
+ * the LightSeq 2020 slides evaluate against max|W| (slide "quantization:
+ * clipping + symmetric").  Per channel n the bound put on level 127 is
+ *   W8_CLIP_FIXED:      bound_n = min( max_k |W[k,n]|, c ),  c = (float)clip_param >= 0
+ *   W8_CLIP_PERCENTILE: bound_n = the r-th smallest |W[k,n]|,
+ *                       r = clamp( ceil(p K), 1, K ) in IEEE double, p = clip_param in (0, 1]
+ * and then s_n = fp16_rne( fp32(bound_n) / 127 ), q = clamp( rne(W / s_n),
+ * -127, 127 ) as in w8_quantize_per_channel: weights beyond the bound land on
+ * +-127.  The output is in the symmetric format (w8_prepack, w8a16_linear).
+ * c = +inf and p = 1 give w8_quantize_per_channel's result bit for bit.
+ * The percentile form finds the order statistic by a four-pass radix
+ * selection on the bit patterns of |w| and streams W five times (the passes
+ * after the first mostly from L2).
+ * Errors: as w8_quantize_per_channel; W8_ERR_SHAPE also for a clip_param
+ * out of range, W8_ERR_DTYPE for an unknown clip_mode.
+ */
+typedef enum { W8_CLIP_FIXED = 0, W8_CLIP_PERCENTILE = 1 } w8_clip_mode;
+
+int w8_quantize_per_channel_clip(const void *W, int w_dtype, int64_t K, int64_t N, int clip_mode,
+                                 double clip_param, int8_t *q, uint16_t *scales, void *stream);
+
+/*
  * w8_prepacked_bytes -- size of the packed weight for a [K, N] q:
  * ceil(N/128) * ceil(K/64) * 8192 bytes (== K*N when K % 64 == 0 and
  * N % 128 == 0).  Returns 0 for K < 1 or N < 1.

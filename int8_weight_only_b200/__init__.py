@@ -18,7 +18,7 @@ import os
 import threading
 
 __all__ = [
-    "W8Error", "load_library", "library_path", "quantize", "quantize_asym", "prepack", "unpack",
+    "W8Error", "load_library", "library_path", "quantize", "quantize_asym", "quantize_clip", "prepack", "unpack",
     "prepacked_bytes", "workspace_bytes", "linear", "linear_asym", "linear_decode_static", "W8A16Linear", "device_status",
     "test_bounded_wait", "STATUS",
 ]
@@ -62,6 +62,7 @@ def load_library():
         vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
         lib.w8_quantize_per_channel.argtypes = [vp, i32, i64, i64, vp, vp, vp]
         lib.w8_quantize_per_channel_asym.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
+        lib.w8_quantize_per_channel_clip.argtypes = [vp, i32, i64, i64, i32, ctypes.c_double, vp, vp, vp]
         lib.w8a16_linear_asym.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp]
         lib.w8_prepacked_bytes.argtypes = [i64, i64]
         lib.w8_prepacked_bytes.restype = sz
@@ -169,6 +170,41 @@ def quantize_asym(W, q=None, scales=None, zeros=None):
         _check(lib.w8_quantize_per_channel_asym(_ptr(W), dt, K, N, _ptr(q), _ptr(scales), _ptr(zeros),
                                                 _stream(W.device)), "w8_quantize_per_channel_asym")
     return q, scales, zeros
+
+
+W8_CLIP_FIXED, W8_CLIP_PERCENTILE = 0, 1
+
+
+def quantize_clip(W, mode, param, q=None, scales=None):
+    """Symmetric int8 quantization of W [K, N] with a clipped bound.
+
+    mode "fixed": bound = min(max|W|, param) per channel; mode "percentile":
+    bound = the ceil(param K)-th smallest |W| per channel.  Returns
+    (q int8 [K, N], scales fp16 [N]) in the format of ``quantize``.
+    """
+    torch = _torch()
+    lib = load_library()
+    _need_cuda(W, "W")
+    modes = {"fixed": W8_CLIP_FIXED, "percentile": W8_CLIP_PERCENTILE}
+    if mode not in modes:
+        raise ValueError("mode must be 'fixed' or 'percentile'")
+    if W.dim() != 2:
+        raise ValueError("W must be [K, N]")
+    if W.dtype == torch.float32:
+        dt = W8_F32
+    elif W.dtype == torch.float16:
+        dt = W8_F16
+    else:
+        raise ValueError("W must be float32 or float16")
+    K, N = W.shape
+    if q is None:
+        q = torch.empty((K, N), dtype=torch.int8, device=W.device)
+    if scales is None:
+        scales = torch.empty((N,), dtype=torch.float16, device=W.device)
+    with torch.cuda.device(W.device):
+        _check(lib.w8_quantize_per_channel_clip(_ptr(W), dt, K, N, modes[mode], float(param), _ptr(q),
+                                                _ptr(scales), _stream(W.device)), "w8_quantize_per_channel_clip")
+    return q, scales
 
 
 def prepack(q, out=None):

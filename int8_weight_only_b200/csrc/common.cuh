@@ -46,6 +46,9 @@ enum WaitSite : unsigned {
     SITE_P2_DFULL = 0x47,
     SITE_P2_DRAIN = 0x48,
     SITE_P2_FIX = 0x49,
+    SITE_CLIP_EMPTY = 0x50,
+    SITE_CLIP_LOAD = 0x51,
+    SITE_CLIP_DRAIN = 0x52,
     SITE_SELFTEST = 0xEE,
 };
 

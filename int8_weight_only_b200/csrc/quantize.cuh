@@ -141,6 +141,7 @@ struct Params {
     int8_t *q;
     uint16_t *scales;
     int8_t *zeros;     // asymmetric form only: [N] zero points
+    float clip;        // symmetric form: bound = min(max|W|, clip); +inf: no clip
     int64_t K;
     int64_t N;
     int kc;            // rows per cluster rank (multiple of the box height)
@@ -339,7 +340,7 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                     for (uint32_t r = 0; r < csize; ++r) lo = fminf(lo, ld_dsmem_f32(mapa_shared(local_lo, r)));
                     asym_params(lo, m, s16, z);
                 } else {
-                    s16 = __float2half_rn(__fdiv_rn(m, 127.0f));
+                    s16 = __float2half_rn(__fdiv_rn(fminf(m, p.clip), 127.0f));
                 }
                 const float sf = __half2float(s16);
                 col_scale[c] = sf;

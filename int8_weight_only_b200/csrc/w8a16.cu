@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <climits>
 #include <mutex>
 
@@ -15,6 +16,7 @@
 #include "prefill2.cuh"
 #include "prepack.cuh"
 #include "quantize.cuh"
+#include "clip.cuh"
 
 namespace {
 
@@ -72,6 +74,8 @@ int device_info(DeviceInfo **out) {
             smem((const void *)quant::quantize_kernel<__half, false>, quant::kSmemBytes);
             smem((const void *)quant::quantize_kernel<float, true>, quant::kSmemBytes);
             smem((const void *)quant::quantize_kernel<__half, true>, quant::kSmemBytes);
+            smem((const void *)clip::percentile_quantize_kernel<float>, clip::kSmemBytes);
+            smem((const void *)clip::percentile_quantize_kernel<__half>, clip::kSmemBytes);
             if (e != cudaSuccess) return W8_ERR_CUDA;
         }
         d.ready = true;
@@ -134,7 +138,7 @@ inline int quantize_cluster(int64_t K, int rows_per_box) {
 
 template <typename T, bool kAsym>
 int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_t K, int64_t N,
-                    int8_t *q, uint16_t *scales, int8_t *zeros, cudaStream_t st) {
+                    int8_t *q, uint16_t *scales, int8_t *zeros, float clip_bound, cudaStream_t st) {
     constexpr int rows = quant::Box<T>::kRows;
     const int C = quantize_cluster(K, rows);
     const int64_t kc = cdiv(cdiv(K, C), rows) * rows;
@@ -179,6 +183,7 @@ int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_
     p.q = q;
     p.scales = scales;
     p.zeros = zeros;
+    p.clip = clip_bound;
     p.K = K;
     p.N = N;
     p.kc = (int)kc;
@@ -210,6 +215,31 @@ int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t 
         cudaGetLastError();
         return W8_ERR_CUDA;
     }
+    return launch_status();
+}
+
+// Percentile clip (clip.cuh): one persistent CTA per SM, panels of 32
+// columns; t = K - r + 1 with r = clamp(ceil(p K), 1, K) in IEEE double.
+template <typename T>
+int launch_percentile(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_t K, int64_t N, double pct,
+                      int8_t *q, uint16_t *scales, cudaStream_t st) {
+    const double rr = std::ceil(pct * (double)K);
+    const int64_t r = rr < 1.0 ? 1 : (rr > (double)K ? K : (int64_t)rr);
+    const int64_t panels = cdiv(N, clip::kPanel);
+    if (panels > INT32_MAX || K > INT32_MAX) return W8_ERR_SHAPE;
+    CUtensorMap map;
+    int rc = make_map_2d(&map, W, dt, (int)sizeof(T), (uint64_t)N, (uint64_t)K, clip::kPanel,
+                         clip::Geo<T>::kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc != W8_OK) return rc;
+    clip::Params p;
+    p.q = q;
+    p.scales = scales;
+    p.K = K;
+    p.N = N;
+    p.t = (int)(K - r + 1);
+    p.panels = (int)panels;
+    const int grid = (int)std::min<int64_t>(panels, d->sms);
+    clip::percentile_quantize_kernel<T><<<grid, clip::kThreads, clip::kSmemBytes, st>>>(map, p);
     return launch_status();
 }
 
@@ -339,7 +369,8 @@ const char *w8_error_string(int status) {
 
 // Both quantization forms: zeros == nullptr selects the symmetric one.
 static int quantize_common(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q, uint16_t *scales,
-                           int8_t *zeros, bool asym, void *stream) {
+                           int8_t *zeros, bool asym, void *stream, float clip_bound = INFINITY,
+                           double percentile = 0.0) {
     if (w_dtype != W8_F32 && w_dtype != W8_F16) return W8_ERR_DTYPE;
     if (K < 1 || N < 0 || N % 8 != 0 || K > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX * 8)
         return W8_ERR_SHAPE;
@@ -358,14 +389,23 @@ static int quantize_common(const void *W, int w_dtype, int64_t K, int64_t N, int
     int rc = device_info(&d);
     if (rc != W8_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (percentile > 0.0) {
+        if (w_dtype == W8_F32)
+            return launch_percentile<float>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, percentile, q, scales, st);
+        return launch_percentile<__half>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, percentile, q, scales, st);
+    }
     if (asym) {
         if (w_dtype == W8_F32)
-            return launch_quantize<float, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, zeros, st);
-        return launch_quantize<__half, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, zeros, st);
+            return launch_quantize<float, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, zeros,
+                                                INFINITY, st);
+        return launch_quantize<__half, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, zeros,
+                                             INFINITY, st);
     }
     if (w_dtype == W8_F32)
-        return launch_quantize<float, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, nullptr, st);
-    return launch_quantize<__half, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, nullptr, st);
+        return launch_quantize<float, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, nullptr,
+                                             clip_bound, st);
+    return launch_quantize<__half, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, nullptr,
+                                          clip_bound, st);
 }
 
 int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
@@ -376,6 +416,20 @@ int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, in
 int w8_quantize_per_channel_asym(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
                                  uint16_t *scales, int8_t *zeros, void *stream) {
     return quantize_common(W, w_dtype, K, N, q, scales, zeros, true, stream);
+}
+
+int w8_quantize_per_channel_clip(const void *W, int w_dtype, int64_t K, int64_t N, int clip_mode,
+                                 double clip_param, int8_t *q, uint16_t *scales, void *stream) {
+    if (clip_mode == W8_CLIP_FIXED) {
+        const float c = (float)clip_param;
+        if (!(c >= 0.0f)) return W8_ERR_SHAPE;   // negative or NaN
+        return quantize_common(W, w_dtype, K, N, q, scales, nullptr, false, stream, c);
+    }
+    if (clip_mode == W8_CLIP_PERCENTILE) {
+        if (!(clip_param > 0.0 && clip_param <= 1.0)) return W8_ERR_SHAPE;
+        return quantize_common(W, w_dtype, K, N, q, scales, nullptr, false, stream, INFINITY, clip_param);
+    }
+    return W8_ERR_DTYPE;
 }
 
 size_t w8_prepacked_bytes(int64_t K, int64_t N) {

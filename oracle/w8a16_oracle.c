@@ -231,7 +231,7 @@ void oracle_linear(const uint16_t *X, const int8_t *q, const uint16_t *scales,
  * 2020 slides evaluate ("fixed range clip" and "percentage clip" against
  * plain max|W|, slide "quantization: clipping + symmetric").  The bound
  * that is put on level 127 is, per channel n:
- *   fixed range:  bound_n = min( max_k |W[k,n]|, c )        (c >= 0)
+ *   fixed range:  bound_n = min( max_k |W[k,n]|, c )        (c >= 0, fp32)
  *   percentage:   bound_n = the r-th smallest |W[k,n]|,
  *                 r = clamp( ceil(p K), 1, K ) in IEEE double  (0 < p <= 1)
  * and then, as in the symmetric quantizer, S = fp16_rne(fp32(bound)/127)
@@ -279,8 +279,9 @@ static void quantize_clip_column(const float *col_vals, int64_t K, int mode, dou
                 bound = mag;
             }
         }
-        if ((double)bound > param) {
-            bound = (float)param;
+        float cf = (float)param;               /* the clip is an fp32 value */
+        if (bound > cf) {
+            bound = cf;
         }
     } else {
         double rr = ceil(param * (double)K);

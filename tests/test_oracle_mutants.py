@@ -52,7 +52,7 @@ MUTANTS = {
     "percentile_rank_off_by_one": ("bound = sort_buf[r - 1];", "bound = sort_buf[r > 1 ? r - 2 : 0];"),
     "percentile_floor_rank": ("double rr = ceil(param * (double)K);", "double rr = floor(param * (double)K);"),
     "percentile_signed_values": ("sort_buf[k] = fabsf(col_vals[k]);", "sort_buf[k] = col_vals[k];"),
-    "fixed_clip_ignored": ("if ((double)bound > param) {", "if (0) {"),
+    "fixed_clip_ignored": ("if (bound > cf) {", "if (0) {"),
     "clip_codes_not_clamped": ("rr = clampf_range(rr, -127.0f, 127.0f);", "rr = clampf_range(rr, -128.0f, 127.0f);"),
     "asym_linear_scale_by_row": ("acc[col] * (double)oracle_f16_to_f32(scales[col])",
                                  "acc[col] * (double)oracle_f16_to_f32(scales[row])"),
