@@ -66,6 +66,11 @@ class Oracle:
         lib.oracle_quantize_clip.argtypes = [vp, ctypes.c_int, i64, i64, ctypes.c_int, ctypes.c_double,
                                              vp, vp, vp, vp]
         lib.oracle_quantize_clip.restype = None
+        lib.oracle_quantize_outliers.argtypes = [vp, ctypes.c_int, i64, i64, ctypes.c_double, vp, vp, vp, vp,
+                                                 vp, vp, vp]
+        lib.oracle_quantize_outliers.restype = None
+        lib.oracle_linear_outliers.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, i64, i64, i64, vp, vp]
+        lib.oracle_linear_outliers.restype = None
         for f in ("oracle_f32_to_f16_array", "oracle_f16_to_f32_array",
                   "oracle_quantize_f32", "oracle_quantize_f16", "oracle_linear",
                   "oracle_quantize_asym_f32", "oracle_quantize_asym_f16", "oracle_linear_asym"):
@@ -177,6 +182,54 @@ class Oracle:
                                       _ptr(buf), _ptr(sbuf))
         return q, s.view(np.float16)
 
+    def quantize_outliers(self, W: np.ndarray, p: float):
+        """Outlier split: per channel, weights with |w| above the
+        ceil(pK)-th smallest magnitude are kept as fp16 (code 0), the rest
+        quantized with that bound.  Returns (q, scales, count int32 [N],
+        rows int32 [N, cap], vals float16 [N, cap]) with cap = K - r."""
+        if W.ndim != 2:
+            raise ValueError("W must be 2-D [K, N]")
+        K, N = W.shape
+        rr = np.ceil(np.float64(p) * np.float64(K))
+        r = int(min(max(rr, 1.0), float(K)))
+        cap = K - r
+        q = np.empty((K, N), dtype=np.int8)
+        s = np.empty(N, dtype=np.uint16)
+        cnt = np.empty(N, dtype=np.int32)
+        rows = np.empty((N, max(cap, 0)), dtype=np.int32)
+        vals = np.empty((N, max(cap, 0)), dtype=np.uint16)
+        buf = np.empty(max(K, 1), dtype=np.float32)
+        sbuf = np.empty(max(K, 1), dtype=np.float32)
+        if W.dtype == np.float32:
+            Wc, f16 = np.ascontiguousarray(W), 0
+        elif W.dtype == np.float16:
+            Wc, f16 = np.ascontiguousarray(W).view(np.uint16), 1
+        else:
+            raise TypeError("W must be float32 or float16")
+        self.lib.oracle_quantize_outliers(_ptr(Wc), f16, K, N, float(p), _ptr(q), _ptr(s), _ptr(cnt),
+                                          _ptr(rows), _ptr(vals), _ptr(buf), _ptr(sbuf))
+        return q, s.view(np.float16), cnt, rows, vals.view(np.float16)
+
+    def linear_outliers(self, X, q, scales, count, rows, vals, bias=None) -> np.ndarray:
+        """Y = X . dequant(q) + X . outliers (+ bias) in fp64 (not rounded)."""
+        M, K = X.shape
+        K2, N = q.shape
+        cap = rows.shape[1]
+        if K2 != K or scales.shape != (N,) or count.shape != (N,) or vals.shape != (N, cap):
+            raise ValueError("shape mismatch")
+        Xc = np.ascontiguousarray(X, dtype=np.float16).view(np.uint16)
+        qc = np.ascontiguousarray(q, dtype=np.int8)
+        sc = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
+        cc = np.ascontiguousarray(count, dtype=np.int32)
+        rc = np.ascontiguousarray(rows, dtype=np.int32)
+        vc = np.ascontiguousarray(vals, dtype=np.float16).view(np.uint16)
+        bc = None if bias is None else np.ascontiguousarray(bias, dtype=np.float16).view(np.uint16)
+        Y = np.empty((M, N), dtype=np.float64)
+        acc = np.empty(max(N, 1), dtype=np.float64)
+        self.lib.oracle_linear_outliers(_ptr(Xc), _ptr(qc), _ptr(sc), _ptr(cc), _ptr(rc), _ptr(vc), cap,
+                                        None if bc is None else _ptr(bc), M, K, N, _ptr(Y), _ptr(acc))
+        return Y
+
     def linear_asym(self, X, q, scales, zeros, bias=None) -> np.ndarray:
         """Y = X . ((q - zeros) o scales) (+ bias) in fp64 (not rounded)."""
         M, K = X.shape
@@ -229,6 +282,14 @@ def linear_asym(X, q, scales, zeros, bias=None):
 
 def quantize_clip(W, mode, param):
     return default().quantize_clip(W, mode, param)
+
+
+def quantize_outliers(W, p):
+    return default().quantize_outliers(W, p)
+
+
+def linear_outliers(X, q, scales, count, rows, vals, bias=None):
+    return default().linear_outliers(X, q, scales, count, rows, vals, bias)
 
 
 def tolerance_ok(y_test: np.ndarray, y_ref: np.ndarray):

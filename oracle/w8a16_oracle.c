@@ -309,6 +309,76 @@ void oracle_quantize_clip(const void *W, int w_is_f16, int64_t K, int64_t N, int
 }
 
 /* ---------------------------------------------------------------------
+ * Outlier split -- the observation of the GOBO page applied to W8A16: the
+ * few largest-magnitude weights of a channel inflate its scale, so they are
+ * kept apart, exactly (as fp16), and the rest is quantized with the scale
+ * of the remaining range.  Per channel n, with bound_n the r-th smallest
+ * |W[k,n]|, r = clamp(ceil(p K), 1, K) in IEEE double (the percentage
+ * clip's bound):
+ *   outliers: every k with |W[k,n]| > bound_n, in increasing k; each kept
+ *             as (k, fp16_rne(W[k,n])) and given the code 0;
+ *   the rest: S = fp16_rne(fp32(bound_n)/127), q = clamp(rne(W/S), -127, 127).
+ * At most cap = K - r weights of a channel are outliers (cap = 0 for p = 1,
+ * the plain symmetric quantizer).  The side list is stored per channel in
+ * cap slots: count[n], rows[n*cap + j], vals[n*cap + j] (unused slots 0).
+ *   Y[m,n] = S_n sum_k X[m,k] q[k,n] + sum_j X[m, rows_j] vals_j + bias_n
+ * ------------------------------------------------------------------- */
+
+void oracle_quantize_outliers(const void *W, int w_is_f16, int64_t K, int64_t N, double p,
+                              int8_t *q, uint16_t *scales, int32_t *count, int32_t *rows,
+                              uint16_t *vals, float *col_buf, float *sort_buf)
+{
+    double rr = ceil(p * (double)K);
+    int64_t r = rr < 1.0 ? 1 : (rr > (double)K ? K : (int64_t)rr);
+    int64_t cap = K - r;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            col_buf[k] = w_is_f16 ? oracle_f16_to_f32(((const uint16_t *)W)[k * N + n])
+                                  : ((const float *)W)[k * N + n];
+            sort_buf[k] = fabsf(col_buf[k]);
+        }
+        qsort(sort_buf, (size_t)K, sizeof(float), compare_floats);
+        float cut = sort_buf[r - 1];
+        codes_for_bound(col_buf, K, cut, q + n, N, &scales[n]);
+        int32_t c = 0;
+        for (int64_t j = 0; j < cap; ++j) {
+            rows[n * cap + j] = 0;
+            vals[n * cap + j] = 0;
+        }
+        for (int64_t k = 0; k < K; ++k) {
+            /* at most K - r magnitudes exceed the r-th smallest, so c < cap
+             * always holds; the test only keeps every write inside the slots */
+            if (fabsf(col_buf[k]) > cut && c < cap) {
+                rows[n * cap + c] = (int32_t)k;
+                vals[n * cap + c] = oracle_f32_to_f16(col_buf[k]);
+                q[k * N + n] = 0;
+                ++c;
+            }
+        }
+        count[n] = c;
+    }
+}
+
+/* Y[M,N] = X . dequant(q) + X . outliers (+ bias), in fp64. */
+void oracle_linear_outliers(const uint16_t *X, const int8_t *q, const uint16_t *scales,
+                            const int32_t *count, const int32_t *rows, const uint16_t *vals,
+                            int64_t cap, const uint16_t *bias, int64_t M, int64_t K, int64_t N,
+                            double *Y, double *acc)
+{
+    oracle_linear(X, q, scales, bias, M, K, N, Y, acc);
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double extra = 0.0;
+            for (int32_t j = 0; j < count[n]; ++j) {
+                extra += (double)oracle_f16_to_f32(X[m * K + rows[n * cap + j]]) *
+                         (double)oracle_f16_to_f32(vals[n * cap + j]);
+            }
+            Y[m * N + n] += extra;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------
  * Asymmetric (affine) per-output-channel int8 quantization -- the variant
  * the LightSeq 2020 slides set against the symmetric one (slide
  * "quantization: clipping + symmetric": a weight is (i - z) S, and the

@@ -54,6 +54,14 @@ MUTANTS = {
     "percentile_signed_values": ("sort_buf[k] = fabsf(col_vals[k]);", "sort_buf[k] = col_vals[k];"),
     "fixed_clip_ignored": ("if (bound > cf) {", "if (0) {"),
     "clip_codes_not_clamped": ("rr = clampf_range(rr, -127.0f, 127.0f);", "rr = clampf_range(rr, -128.0f, 127.0f);"),
+    # outlier split
+    "outlier_at_or_above_bound": ("if (fabsf(col_buf[k]) > cut && c < cap) {",
+                                  "if (fabsf(col_buf[k]) >= cut && c < cap) {"),
+    "outlier_code_kept": ("                q[k * N + n] = 0;\n", ""),
+    "outlier_value_not_added": ("            Y[m * N + n] += extra;", "            Y[m * N + n] += 0.0 * extra;"),
+    "outlier_row_as_token": ("X[m * K + rows[n * cap + j]]", "X[rows[n * cap + j] % M * K + m % K]"),
+    "outlier_value_fp32_truncated": ("vals[n * cap + c] = oracle_f32_to_f16(col_buf[k]);",
+                                     "vals[n * cap + c] = (uint16_t)(oracle_f32_to_f16(col_buf[k]) & 0xFFFCu);"),
     "asym_linear_scale_by_row": ("acc[col] * (double)oracle_f16_to_f32(scales[col])",
                                  "acc[col] * (double)oracle_f16_to_f32(scales[row])"),
 }

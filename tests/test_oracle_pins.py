@@ -462,6 +462,76 @@ def pin_fixed_clip_scale_and_codes(orc):
     assert s2[5] == ss[0] and np.array_equal(q2[:, 5], qs[:, 0])
 
 
+# ---------------------------------------------------------------- outlier split
+# weights above the percentage-clip bound kept apart as fp16, code 0; the
+# rest quantized with that bound.
+
+def pin_outliers_p_one_is_the_symmetric_quantizer(orc):
+    W = synthetic.weights(300, 40, SEED, 151, outlier_frac=0.01)
+    q, s, cnt, rows, vals = orc.quantize_outliers(W, 1.0)
+    q0, s0 = orc.quantize(W)
+    assert rows.shape == (40, 0) and not cnt.any()
+    assert np.array_equal(q, q0) and np.array_equal(s.view(np.uint16), s0.view(np.uint16))
+    X = synthetic.activations(3, 300, SEED, 152)
+    assert np.array_equal(orc.linear_outliers(X, q, s, cnt, rows, vals), orc.linear(X, q0, s0))
+
+
+def pin_outliers_are_the_largest_magnitudes(orc):
+    # |w| = delta, 2 delta, ..., K delta per column (shuffled, random signs):
+    # the outliers are exactly the K - r largest, in increasing row order
+    rng = np.random.default_rng(45)
+    K, N, delta = 400, 10, 2.0 ** -10
+    W = np.empty((K, N), dtype=np.float32)
+    for n in range(N):
+        W[:, n] = rng.permutation(np.arange(1, K + 1)) * delta * rng.choice([-1.0, 1.0], K)
+    for p, r in ((0.99, 396), (0.9501, 381)):
+        q, s, cnt, rows, vals = orc.quantize_outliers(W, p)
+        cap = K - r
+        assert rows.shape == (N, cap) and np.all(cnt == cap)
+        for n in range(N):
+            want = np.sort(np.argsort(np.abs(W[:, n]))[r:])
+            assert np.array_equal(rows[n], want)
+            assert np.array_equal(vals[n].astype(np.float32), W[want, n])   # exact in fp16
+            assert not q[want, n].any()
+        assert np.all(s == np.float16(np.float32(r * delta) / np.float32(127.0)))
+
+
+def pin_outlier_split_reconstructs_the_weight(orc):
+    K, N = 512, 64
+    W = synthetic.weights(K, N, SEED, 153, outlier_frac=0.01)
+    for p in (0.999, 0.99, 0.95):
+        q, s, cnt, rows, vals = orc.quantize_outliers(W, p)
+        deq = q.astype(np.float64) * s.astype(np.float64)
+        for n in range(N):
+            deq[rows[n, :cnt[n]], n] += vals[n, :cnt[n]].astype(np.float64)
+            assert np.all(np.diff(rows[n, :cnt[n]]) > 0) and not rows[n, cnt[n]:].any()
+        is_out = np.zeros((K, N), dtype=bool)
+        for n in range(N):
+            is_out[rows[n, :cnt[n]], n] = True
+        err = np.abs(deq - W.astype(np.float64))
+        sf = s.astype(np.float64)
+        assert np.all(err[~is_out] <= (0.5 + 2.0 ** -10) * np.broadcast_to(sf, (K, N))[~is_out])
+        assert np.all(err[is_out] <= 2.0 ** -11 * np.abs(W.astype(np.float64))[is_out])
+
+
+def pin_outlier_linear_unit_rows(orc):
+    K, N = 200, 24
+    W = synthetic.weights(K, N, SEED, 154, outlier_frac=0.02)
+    q, s, cnt, rows, vals = orc.quantize_outliers(W, 0.97)
+    b = synthetic.bias(N, SEED, 155)
+    ks = [int(rows[0, 0]), 5, 199]
+    X = np.zeros((len(ks), K), dtype=np.float16)
+    X[np.arange(len(ks)), ks] = 1.0
+    Y = orc.linear_outliers(X, q, s, cnt, rows, vals, b)
+    for i, k in enumerate(ks):
+        want = q[k].astype(np.float64) * s.astype(np.float64) + b.astype(np.float64)
+        for n in range(N):
+            hit = np.nonzero(rows[n, :cnt[n]] == k)[0]
+            if hit.size:
+                want[n] += float(vals[n, hit[0]])
+        assert np.array_equal(Y[i], want)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
