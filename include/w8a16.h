@@ -134,6 +134,43 @@ int w8_quantize_per_channel_clip(const void *W, int w_dtype, int64_t K, int64_t 
                                  double clip_param, int8_t *q, uint16_t *scales, void *stream);
 
 /*
+ * Outlier split -- the observation of the GOBO page (a few large weights
+ * inflate the scale; keep them apart, exactly) applied to W8A16.  Per channel
+ * n, with bound_n = the r-th smallest |W[k,n]|, r = clamp(ceil(p K), 1, K) in
+ * IEEE double (the percentage clip's bound):
+ *   outliers: every k with |W[k,n]| > bound_n, kept as (k, fp16_rne(W[k,n]))
+ *             in increasing k, with code 0;
+ *   the rest: s_n = fp16_rne(fp32(bound_n)/127), q = clamp(rne(W/s_n), -127, 127).
+ * At most cap = K - r weights of a channel are outliers.  The side list has
+ * cap slots per channel: o_count [N] int32, o_rows [N][cap] int32, o_vals
+ * [N][cap] fp16; unused slots are 0.  p = 1 gives cap = 0 and the plain
+ * symmetric quantizer.
+ *
+ * w8_outlier_capacity -- cap for (K, p); 0 for arguments out of range.
+ * w8_quantize_per_channel_outliers -- the split above.  0 < p <= 1; cap must
+ *   not exceed 64 (W8_ERR_LIMIT), i.e. p >= 1 - 64/K roughly; o_rows and
+ *   o_vals may be NULL when cap == 0.  Bit-exact; other arguments and errors
+ *   as w8_quantize_per_channel.
+ * w8a16_linear_outliers -- Y = X . dequant(q) + X . outliers (+ bias):
+ *   Y[m,n] = s_n sum_k X[m,k] q[k,n] + sum_j X[m, rows_j] vals_j + bias_n,
+ *   the outlier products added in fp32 before the single rounding to fp16.
+ *   packed/scales from w8_prepack of the split's q; o_cap the cap it was made
+ *   with.  The workspace must hold w8a16_linear_outliers_workspace_bytes(M,
+ *   K, N) bytes (for M > 64 it also holds X transposed, written by the call).
+ *   Accuracy, stream ordering and errors as w8a16_linear; W8_ERR_LIMIT for
+ *   o_cap > 64.
+ */
+size_t w8_outlier_capacity(int64_t K, double p);
+int w8_quantize_per_channel_outliers(const void *W, int w_dtype, int64_t K, int64_t N, double p, int8_t *q,
+                                     uint16_t *scales, int32_t *o_count, int32_t *o_rows, uint16_t *o_vals,
+                                     void *stream);
+size_t w8a16_linear_outliers_workspace_bytes(int64_t M, int64_t K, int64_t N);
+int w8a16_linear_outliers(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
+                          const int32_t *o_count, const int32_t *o_rows, const uint16_t *o_vals, int64_t o_cap,
+                          const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/*
  * w8_prepacked_bytes -- size of the packed weight for a [K, N] q:
  * ceil(N/128) * ceil(K/64) * 8192 bytes (== K*N when K % 64 == 0 and
  * N % 128 == 0).  Returns 0 for K < 1 or N < 1.

@@ -18,8 +18,8 @@ import os
 import threading
 
 __all__ = [
-    "W8Error", "load_library", "library_path", "quantize", "quantize_asym", "quantize_clip", "prepack", "unpack",
-    "prepacked_bytes", "workspace_bytes", "linear", "linear_asym", "linear_decode_static", "W8A16Linear", "device_status",
+    "W8Error", "load_library", "library_path", "quantize", "quantize_asym", "quantize_clip", "quantize_outliers", "prepack", "unpack",
+    "prepacked_bytes", "workspace_bytes", "linear", "linear_asym", "linear_outliers", "linear_decode_static", "W8A16Linear", "device_status",
     "test_bounded_wait", "STATUS",
 ]
 
@@ -63,6 +63,13 @@ def load_library():
         lib.w8_quantize_per_channel.argtypes = [vp, i32, i64, i64, vp, vp, vp]
         lib.w8_quantize_per_channel_asym.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
         lib.w8_quantize_per_channel_clip.argtypes = [vp, i32, i64, i64, i32, ctypes.c_double, vp, vp, vp]
+        lib.w8_outlier_capacity.argtypes = [i64, ctypes.c_double]
+        lib.w8_outlier_capacity.restype = sz
+        lib.w8_quantize_per_channel_outliers.argtypes = [vp, i32, i64, i64, ctypes.c_double, vp, vp, vp, vp, vp,
+                                                         vp]
+        lib.w8a16_linear_outliers_workspace_bytes.argtypes = [i64, i64, i64]
+        lib.w8a16_linear_outliers_workspace_bytes.restype = sz
+        lib.w8a16_linear_outliers.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp, i64, i64, i64, vp, sz, vp]
         lib.w8a16_linear_asym.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp]
         lib.w8_prepacked_bytes.argtypes = [i64, i64]
         lib.w8_prepacked_bytes.restype = sz
@@ -205,6 +212,62 @@ def quantize_clip(W, mode, param, q=None, scales=None):
         _check(lib.w8_quantize_per_channel_clip(_ptr(W), dt, K, N, modes[mode], float(param), _ptr(q),
                                                 _ptr(scales), _stream(W.device)), "w8_quantize_per_channel_clip")
     return q, scales
+
+
+def quantize_outliers(W, p):
+    """Outlier split of W [K, N]: per channel the weights above the
+    ceil(pK)-th smallest magnitude are kept as fp16 (code 0); the rest is
+    quantized with that bound.  Returns (q int8 [K, N], scales fp16 [N],
+    count int32 [N], rows int32 [N, cap], vals fp16 [N, cap])."""
+    torch = _torch()
+    lib = load_library()
+    _need_cuda(W, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be [K, N]")
+    if W.dtype == torch.float32:
+        dt = W8_F32
+    elif W.dtype == torch.float16:
+        dt = W8_F16
+    else:
+        raise ValueError("W must be float32 or float16")
+    K, N = W.shape
+    cap = int(lib.w8_outlier_capacity(K, float(p)))
+    dev = W.device
+    q = torch.empty((K, N), dtype=torch.int8, device=dev)
+    scales = torch.empty((N,), dtype=torch.float16, device=dev)
+    count = torch.empty((N,), dtype=torch.int32, device=dev)
+    rows = torch.empty((N, cap), dtype=torch.int32, device=dev)
+    vals = torch.empty((N, cap), dtype=torch.float16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib.w8_quantize_per_channel_outliers(_ptr(W), dt, K, N, float(p), _ptr(q), _ptr(scales),
+                                                    _ptr(count), _ptr(rows) if cap else None,
+                                                    _ptr(vals) if cap else None, _stream(dev)),
+               "w8_quantize_per_channel_outliers")
+    return q, scales, count, rows, vals
+
+
+def linear_outliers(X, packed, scales, count, rows, vals, bias=None, out=None, workspace=None):
+    """Y [M, N] fp16 = X . dequant(q) + X . outliers (+ bias), for the
+    output of quantize_outliers (q prepacked)."""
+    torch = _torch()
+    lib = load_library()
+    _need_cuda(X, "X")
+    if X.dim() != 2 or X.dtype != torch.float16:
+        raise ValueError("X must be [M, K] float16")
+    M, K = X.shape
+    N = scales.shape[0]
+    cap = rows.shape[1]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    with torch.cuda.device(X.device):
+        need = int(lib.w8a16_linear_outliers_workspace_bytes(M, K, N))
+        ws = workspace if workspace is not None else _workspace(X.device, need)
+        ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+        _check(lib.w8a16_linear_outliers(_ptr(X), _ptr(packed), _ptr(scales), _ptr(count),
+                                         _ptr(rows) if cap else None, _ptr(vals) if cap else None, cap, _ptr(bias),
+                                         _ptr(out), M, K, N, _ptr(ws), ws_bytes, _stream(X.device)),
+               "w8a16_linear_outliers")
+    return out
 
 
 def prepack(q, out=None):

@@ -42,6 +42,12 @@ struct Geo {
     static constexpr int kRows = kBoxBytes / kRowBytes;   // 128 fp32 or 256 fp16 rows
 };
 
+// Outlier split (the GOBO page's observation applied here): the weights
+// strictly above the bound are kept apart as (row, fp16 value) in a side
+// list of `cap` slots per channel, rows increasing, unused slots 0, and get
+// the code 0.  At most t - 1 = cap weights of a channel exceed the bound.
+constexpr int kMaxOutliers = 64;
+
 struct Params {
     int8_t *q;
     uint16_t *scales;
@@ -49,6 +55,11 @@ struct Params {
     int64_t N;
     int t;         // rank from the top: the bound is the t-th largest |w|
     int panels;    // ceil(N / 32)
+    // outlier split only
+    int32_t *o_count;    // [N]
+    int32_t *o_rows;     // [N][cap]
+    uint16_t *o_vals;    // [N][cap] fp16
+    int cap;             // t - 1 <= kMaxOutliers
 };
 
 __device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
@@ -66,7 +77,7 @@ __device__ __forceinline__ float load_elem<__half>(const uint8_t *p) {
 
 // grid = persistent CTAs, kThreads threads, kSmemBytes dynamic shared
 // memory.  tmap_w: W [K, N], box 32 columns x Geo<T>::kRows rows, no swizzle.
-template <typename T>
+template <typename T, bool kOut>
 __global__ void __launch_bounds__(kThreads, 1)
 percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
     using G = Geo<T>;
@@ -78,6 +89,10 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
     __shared__ uint32_t col_prefix[kPanel];   // chosen high bytes of the bound's pattern
     __shared__ int col_rem[kPanel];           // rank still to find within them
     __shared__ float col_scale[kPanel], col_inv[kPanel];
+    // outlier split: this panel's side lists, filled in the code pass
+    __shared__ int o_n[kOut ? kPanel : 1];
+    __shared__ int32_t o_row[kOut ? kPanel : 1][kOut ? kMaxOutliers : 1];
+    __shared__ uint16_t o_val[kOut ? kPanel : 1][kOut ? kMaxOutliers : 1];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -133,6 +148,7 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
         if (c < kPanel) {
             col_prefix[c] = 0;
             col_rem[c] = p.t;
+            if constexpr (kOut) o_n[c] = 0;
         }
         for (int i = c; i < kPanel * kBinStride; i += kConsumers) hist[i] = 0;
         for (int pass = 0; pass < kPasses; ++pass) {
@@ -141,7 +157,8 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
             if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
             const int shift = 24 - 8 * pass;   // byte of the pattern this pass histograms
             const uint32_t hi_mask = pass == 0 ? 0u : ~((1u << (shift + 8)) - 1u);
-            const uint32_t prefix = pass < 4 ? col_prefix[lane] : 0u;
+            // pass 4: col_prefix holds the bound's pattern
+            const uint32_t prefix = col_prefix[lane];
             const float sc = pass == 4 ? col_scale[lane] : 0.0f;
             const float inv = pass == 4 ? col_inv[lane] : 0.0f;
             const int64_t n = (int64_t)panel * kPanel + lane;
@@ -161,6 +178,16 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
                             bool sure;
                             int code = quant::quantize_fast(v, inv, sure);
                             if (!sure) code = quant::quantize_exact(v, sc);
+                            if constexpr (kOut) {
+                                if (abs_bits(v) > prefix) {   // |w| above the bound
+                                    const int j = atomicAdd(&o_n[lane], 1);
+                                    if (j < kMaxOutliers) {
+                                        o_row[lane][j] = (int32_t)k;
+                                        o_val[lane][j] = __half_as_ushort(__float2half_rn(v));
+                                    }
+                                    code = 0;
+                                }
+                            }
                             p.q[k * p.N + n] = (int8_t)code;
                         }
                     }
@@ -169,7 +196,37 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
                 if (ok && lane == 0) mbar_arrive(&empty[s]);
                 if (++s == kStages) { s = 0; ph ^= 1u; }
             }
-            if (pass == 4) break;
+            if (pass == 4) {
+                if constexpr (kOut) {
+                    // every outlier of the panel is listed: sort each column's
+                    // list by row (the order the warps met them varies) and
+                    // store it, unused slots 0
+                    if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
+                    const int64_t nn = (int64_t)panel * kPanel + c;
+                    if (c < kPanel && nn < p.N) {
+                        const int cnt = min(o_n[c], p.cap);
+                        for (int a = 1; a < cnt; ++a) {
+                            const int32_t r0 = o_row[c][a];
+                            const uint16_t v0 = o_val[c][a];
+                            int b2 = a - 1;
+                            for (; b2 >= 0 && o_row[c][b2] > r0; --b2) {
+                                o_row[c][b2 + 1] = o_row[c][b2];
+                                o_val[c][b2 + 1] = o_val[c][b2];
+                            }
+                            o_row[c][b2 + 1] = r0;
+                            o_val[c][b2 + 1] = v0;
+                        }
+                        p.o_count[nn] = cnt;
+                        for (int j = 0; j < p.cap; ++j) {
+                            p.o_rows[nn * p.cap + j] = j < cnt ? o_row[c][j] : 0;
+                            p.o_vals[nn * p.cap + j] = j < cnt ? o_val[c][j] : (uint16_t)0;
+                        }
+                    }
+                    // the lists are read before the next panel resets them
+                    if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
+                }
+                break;
+            }
             // the histogram is complete
             if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
             if (c < kPanel) {

@@ -76,6 +76,13 @@ struct Params {
     uint16_t *Y;
     int *counters;
     float *partials;
+    // outlier split (all null otherwise): Y += X[:, rows] . vals per channel
+    const uint16_t *X;           // [M, K] fp16, the activations
+    const int32_t *o_count;      // [N]
+    const int32_t *o_rows;       // [N][o_cap]
+    const uint16_t *o_vals;      // [N][o_cap] fp16
+    int o_cap;
+    int64_t K;
     int M;
     int64_t N;
     int KB;        // ceil(K / 64)
@@ -119,12 +126,29 @@ __device__ __forceinline__ void store_y(const Params &p, uint32_t b, int warp, i
         if (n >= p.N) continue;
         const float s = __half2float(__ushort_as_half(p.scales[n]));
         const float bb = p.bias ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
+        // outlier split: the kept weights' products, added before rounding
+        float extra[MT][2] = {};
+        if (p.o_count) {
+            const int cnt = p.o_count[n];
+            for (int j = 0; j < cnt; ++j) {
+                const int64_t k = p.o_rows[n * p.o_cap + j];
+                const float v = __half2float(__ushort_as_half(p.o_vals[n * p.o_cap + j]));
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int m = 8 * mt + 2 * t + e;
+                        if (m < p.M) extra[mt][e] = fmaf(__half2float(__ushort_as_half(p.X[m * p.K + k])), v,
+                                                         extra[mt][e]);
+                    }
+            }
+        }
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int m = 8 * mt + 2 * t + e;
-                if (m < p.M) p.Y[(int64_t)m * p.N + n] = out_f16(acc[mt][2 * half + e], s, bb);
+                if (m < p.M) p.Y[(int64_t)m * p.N + n] = out_f16(acc[mt][2 * half + e], s, bb + extra[mt][e]);
             }
         }
     }

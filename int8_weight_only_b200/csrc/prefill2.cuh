@@ -98,7 +98,41 @@ struct Params {
     int tiles;     // ceil(NB/2) * TT pair tiles
     int dp_tiles;  // tiles [0, dp_tiles) run whole, round robin
     int sk_iters;  // K steps of tiles [dp_tiles, tiles), split evenly
+    // outlier split (kMode == kOutliers): Y += X[:, rows] . vals per channel
+    const uint16_t *XT;          // [K][Mp] fp16: X transposed, zero for m >= M
+    int64_t Mp;                  // multiple of kBT
+    const int32_t *o_count;      // [N]
+    const int32_t *o_rows;       // [N][o_cap]
+    const uint16_t *o_vals;      // [N][o_cap] fp16
+    int o_cap;
+    float *o_extra;              // per CTA kExtraFloats: the current tile's bias + outlier terms
 };
+
+// Outlier term of one CTA's share of a tile, written while its MMAs run and
+// read back in the drain: [256 epilogue threads][128 tokens] fp32.
+constexpr int kExtraFloats = 32 * kEpiWarps * 128;
+
+// Code forms the converters and the epilogue handle.
+constexpr int kSym = 0;        // symmetric codes
+constexpr int kZeroPoint = 1;  // asymmetric codes: the converters widen to q - z
+constexpr int kOutliers = 2;   // symmetric codes plus a sparse fp16 side list
+
+// X^T for the outlier term: XT[k][m] = X[m][k] for m < M, 0 up to Mp.
+// grid (ceil(K/32), Mp/32), 32 x 8 threads.
+__global__ void transpose_x_kernel(const uint16_t *__restrict__ X, uint16_t *__restrict__ XT, int M, int64_t K,
+                                   int64_t Mp) {
+    __shared__ uint16_t tile[32][33];
+    const int64_t k0 = (int64_t)blockIdx.x * 32, m0 = (int64_t)blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int64_t m = m0 + i, k = k0 + threadIdx.x;
+        tile[i][threadIdx.x] = (m < M && k < K) ? X[m * K + k] : (uint16_t)0;
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int64_t k = k0 + i, m = m0 + threadIdx.x;
+        if (k < K) XT[k * Mp + m] = tile[threadIdx.x][i];
+    }
+}
 
 // First stream-K step of pair q (steps numbered from tile dp_tiles' first).
 // The host keeps tiles, sk_iters and sk_iters x pairs below 2^31.
@@ -204,8 +238,7 @@ __device__ __forceinline__ void stream_k_share(float *partials, int *counters, u
 #pragma unroll
         for (int cchunk = 0; cchunk < 4; ++cchunk) {
             uint32_t v[32];
-            tmem_ld_32x32b_x32(lane_addr + 32 * cchunk, v);
-            tmem_wait_ld();
+            tmem_load_32(lane_addr + 32 * cchunk, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) __stcg(mine + (32 * cchunk + i) * kBNc, __uint_as_float(v[i]));
         }
@@ -235,8 +268,7 @@ __device__ __forceinline__ void stream_k_share(float *partials, int *counters, u
             for (int j = j_first; j <= j_last; ++j) {
                 uint32_t v[32];
                 if (j == pair0 && sg.final) {
-                    tmem_ld_32x32b_x32(lane_addr + 32 * cchunk, v);
-                    tmem_wait_ld();
+                    tmem_load_32(lane_addr + 32 * cchunk, v);
                 } else {
                     const float *src = part_of(j) + 32 * cchunk * kBNc;
 #pragma unroll
@@ -269,9 +301,11 @@ __device__ __forceinline__ void stream_k_share(float *partials, int *counters, u
 // grid = 2 x pairs CTAs, cluster dims (2, 1, 1), kThreads threads,
 // kSmemBytes dynamic shared memory.  tmap_x: X [M, K] fp16, box {64, 128},
 // 128-byte swizzle.
-// kZp: asymmetric codes -- the converters widen every weight to q - z_n
-// (exact in fp16) instead of q; nothing else changes.
-template <bool kSplit, bool kZp>
+// kMode == kZeroPoint: the converters widen every weight to q - z_n (exact
+// in fp16) instead of q.  kMode == kOutliers: the epilogue adds each
+// channel's kept weights times the matching X columns before rounding (no
+// K split with it).
+template <bool kSplit, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -436,7 +470,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         while (ok && sched.next(sg)) {
             const bool valid = (sg.tile / p.TT) * 2 + rank < p.NB;
             uint32_t zc = 0x64806480u;   // 1152 + z of this thread's channel
-            if constexpr (kZp) {
+            if constexpr (kMode == kZeroPoint) {
                 const int64_t n = ((int64_t)(sg.tile / p.TT) * 2 + rank) * kBNc + r;
                 if (valid && n < p.N) zc = zp_bias2(p.zeros[n]);
             }
@@ -468,7 +502,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                         const uint32_t w[4] = {c[t][i].x, c[t][i].y, c[t][i].z, c[t][i].w};
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            if constexpr (kZp) {
+                            if constexpr (kMode == kZeroPoint) {
                                 v[8 * i + 2 * j] = unbias2_by(widen_lo2(w[j]), zc);
                                 v[8 * i + 2 * j + 1] = unbias2_by(widen_hi2(w[j]), zc);
                             } else {
@@ -497,6 +531,41 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         Sched sched(pair0, pstep, p.dp_tiles, p.sk_iters, p.KS);
         Seg sg;
         for (; sched.next(sg); ++it) {
+            if constexpr (kMode == kOutliers) {
+                // this tile's bias + outlier terms, formed while its MMAs run
+                // (the gathers from X^T are off the accumulator's path)
+                const int64_t nb = ((int64_t)(sg.tile / p.TT) * 2 + rank) * kBNc + r;
+                const int mb = (int)(sg.tile % p.TT) * kBT + 128 * half;
+                const bool nb_ok = nb < p.N;
+                const float bb = (nb_ok && p.bias) ? __half2float(__ushort_as_half(p.bias[nb])) : 0.0f;
+                const int cnt = nb_ok ? p.o_count[nb] : 0;
+                float4 *dst = reinterpret_cast<float4 *>(p.o_extra + (int64_t)blockIdx.x * kExtraFloats +
+                                                         (threadIdx.x - 256) * 128);
+                for (int cchunk = 0; cchunk < 4; ++cchunk) {
+                    float ex[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ex[i] = bb;
+                    for (int j = 0; j < cnt; ++j) {
+                        const int64_t k = p.o_rows[nb * p.o_cap + j];
+                        const float ov = __half2float(__ushort_as_half(p.o_vals[nb * p.o_cap + j]));
+                        const uint4 *src = reinterpret_cast<const uint4 *>(p.XT + k * p.Mp + mb + 32 * cchunk);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint4 xv = src[u];
+                            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const __half2 x2 = *reinterpret_cast<const __half2 *>(&xw[h]);
+                                ex[8 * u + 2 * h] = fmaf(__low2float(x2), ov, ex[8 * u + 2 * h]);
+                                ex[8 * u + 2 * h + 1] = fmaf(__high2float(x2), ov, ex[8 * u + 2 * h + 1]);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        dst[8 * cchunk + u] = make_float4(ex[4 * u], ex[4 * u + 1], ex[4 * u + 2], ex[4 * u + 3]);
+                }
+            }
             const bool got = warp_all(mbar_wait(&d_full, it & 1, SITE_P2_DFULL));
             if constexpr (kSplit) {
                 // all epilogue warps give up together: the stream-K share
@@ -512,19 +581,40 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             const bool n_ok = n < p.N;
             const float sc = n_ok ? __half2float(__ushort_as_half(p.scales[n])) : 0.0f;
             const float bi = (n_ok && p.bias) ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
+            const int m0 = tb * kBT + 128 * half;
             if (sg.slot < 0) {
-                const int m0 = tb * kBT + 128 * half;
                 uint32_t y2[64];
 #pragma unroll
                 for (int cchunk = 0; cchunk < 4; ++cchunk) {
                     uint32_t v[32];
-                    tmem_ld_32x32b_x32(lane_addr + 32 * cchunk, v);
-                    tmem_wait_ld();
+                    float ex[32];   // outlier form: bias + outlier terms of these tokens
+                    if constexpr (kMode == kOutliers) {
+                        const float4 *srcx = reinterpret_cast<const float4 *>(
+                            p.o_extra + (int64_t)blockIdx.x * kExtraFloats + (threadIdx.x - 256) * 128 + 32 * cchunk);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const __half2 hv = __floats2half2_rn(fmaf(__uint_as_float(v[2 * i]), sc, bi),
-                                                             fmaf(__uint_as_float(v[2 * i + 1]), sc, bi));
-                        y2[16 * cchunk + i] = *reinterpret_cast<const uint32_t *>(&hv);
+                        for (int u = 0; u < 8; ++u) {
+                            const float4 e4 = srcx[u];
+                            ex[4 * u] = e4.x;
+                            ex[4 * u + 1] = e4.y;
+                            ex[4 * u + 2] = e4.z;
+                            ex[4 * u + 3] = e4.w;
+                        }
+                    }
+                    tmem_load_32(lane_addr + 32 * cchunk, v);
+                    if constexpr (kMode == kOutliers) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const __half2 hv = __floats2half2_rn(fmaf(__uint_as_float(v[2 * i]), sc, ex[2 * i]),
+                                                                 fmaf(__uint_as_float(v[2 * i + 1]), sc, ex[2 * i + 1]));
+                            y2[16 * cchunk + i] = *reinterpret_cast<const uint32_t *>(&hv);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const __half2 hv = __floats2half2_rn(fmaf(__uint_as_float(v[2 * i]), sc, bi),
+                                                                 fmaf(__uint_as_float(v[2 * i + 1]), sc, bi));
+                            y2[16 * cchunk + i] = *reinterpret_cast<const uint32_t *>(&hv);
+                        }
                     }
                 }
                 tc_fence_before();
@@ -538,7 +628,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                         if (m + 1 < p.M) p.Y[(int64_t)(m + 1) * p.N + n] = (uint16_t)(y2[i] >> 16);
                     }
                 }
-            } else if constexpr (kSplit) {
+            } else if constexpr (kSplit && kMode != kOutliers) {
                 stream_k_share(p.partials, p.counters, p.Y, p.M, p.N, p.dp_tiles, p.sk_iters, p.KS, sg, pair0,
                                pstep, tmem, rank, warp, lane, &fix_last, leader(&d_empty), sc, bi, n_ok, n, tb);
             }

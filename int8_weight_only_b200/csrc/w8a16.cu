@@ -66,16 +66,19 @@ int device_info(DeviceInfo **out) {
             smem((const void *)decode::decode_kernel<2, true>, decode::Cfg<2>::kSmemBytes);
             smem((const void *)decode::decode_kernel<4, true>, decode::Cfg<4>::kSmemBytes);
             smem((const void *)decode::decode_kernel<8, true>, decode::Cfg<8>::kSmemBytes);
-            smem((const void *)prefill2::prefill2_kernel<false, false>, prefill2::kSmemBytes);
-            smem((const void *)prefill2::prefill2_kernel<true, false>, prefill2::kSmemBytes);
-            smem((const void *)prefill2::prefill2_kernel<false, true>, prefill2::kSmemBytes);
-            smem((const void *)prefill2::prefill2_kernel<true, true>, prefill2::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<false, prefill2::kSym>, prefill2::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<true, prefill2::kSym>, prefill2::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<false, prefill2::kZeroPoint>, prefill2::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<true, prefill2::kZeroPoint>, prefill2::kSmemBytes);
+            smem((const void *)prefill2::prefill2_kernel<false, prefill2::kOutliers>, prefill2::kSmemBytes);
             smem((const void *)quant::quantize_kernel<float, false>, quant::kSmemBytes);
             smem((const void *)quant::quantize_kernel<__half, false>, quant::kSmemBytes);
             smem((const void *)quant::quantize_kernel<float, true>, quant::kSmemBytes);
             smem((const void *)quant::quantize_kernel<__half, true>, quant::kSmemBytes);
-            smem((const void *)clip::percentile_quantize_kernel<float>, clip::kSmemBytes);
-            smem((const void *)clip::percentile_quantize_kernel<__half>, clip::kSmemBytes);
+            smem((const void *)clip::percentile_quantize_kernel<float, false>, clip::kSmemBytes);
+            smem((const void *)clip::percentile_quantize_kernel<__half, false>, clip::kSmemBytes);
+            smem((const void *)clip::percentile_quantize_kernel<float, true>, clip::kSmemBytes);
+            smem((const void *)clip::percentile_quantize_kernel<__half, true>, clip::kSmemBytes);
             if (e != cudaSuccess) return W8_ERR_CUDA;
         }
         d.ready = true;
@@ -220,11 +223,16 @@ int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t 
 
 // Percentile clip (clip.cuh): one persistent CTA per SM, panels of 32
 // columns; t = K - r + 1 with r = clamp(ceil(p K), 1, K) in IEEE double.
-template <typename T>
-int launch_percentile(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_t K, int64_t N, double pct,
-                      int8_t *q, uint16_t *scales, cudaStream_t st) {
+int64_t percentile_rank(int64_t K, double pct) {
     const double rr = std::ceil(pct * (double)K);
-    const int64_t r = rr < 1.0 ? 1 : (rr > (double)K ? K : (int64_t)rr);
+    return rr < 1.0 ? 1 : (rr > (double)K ? K : (int64_t)rr);
+}
+
+template <typename T, bool kOut>
+int launch_percentile(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_t K, int64_t N, double pct,
+                      int8_t *q, uint16_t *scales, int32_t *o_count, int32_t *o_rows, uint16_t *o_vals,
+                      cudaStream_t st) {
+    const int64_t r = percentile_rank(K, pct);
     const int64_t panels = cdiv(N, clip::kPanel);
     if (panels > INT32_MAX || K > INT32_MAX) return W8_ERR_SHAPE;
     CUtensorMap map;
@@ -238,15 +246,28 @@ int launch_percentile(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int6
     p.N = N;
     p.t = (int)(K - r + 1);
     p.panels = (int)panels;
+    p.o_count = o_count;
+    p.o_rows = o_rows;
+    p.o_vals = o_vals;
+    p.cap = (int)(K - r);
     const int grid = (int)std::min<int64_t>(panels, d->sms);
-    clip::percentile_quantize_kernel<T><<<grid, clip::kThreads, clip::kSmemBytes, st>>>(map, p);
+    clip::percentile_quantize_kernel<T, kOut><<<grid, clip::kThreads, clip::kSmemBytes, st>>>(map, p);
     return launch_status();
 }
 
 // Tensor-core linear for M > 64 on CTA pairs (prefill2.cuh).
+// Outlier side list of a linear call (all null when there is none).
+struct Outliers {
+    const int32_t *count = nullptr;
+    const int32_t *rows = nullptr;
+    const uint16_t *vals = nullptr;
+    int64_t cap = 0;
+    uint16_t *xt = nullptr;   // workspace for X^T (tensor-core path)
+};
+
 int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
                     const int8_t *zeros, const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
-                    float *partials, int *counters, cudaStream_t st) {
+                    float *partials, int *counters, const Outliers &o, cudaStream_t st) {
     CUtensorMap map;
     int rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
                          prefill2::kBTc, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -269,6 +290,13 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
     // 32-bit work counts (a 2^31-tile output would not fit in device memory)
     if (tiles >= INT32_MAX / 2 || (int64_t)p.KS * 2 * d->sms >= INT32_MAX) return W8_ERR_SHAPE;
     p.tiles = (int)tiles;
+    p.XT = o.xt;
+    p.Mp = cdiv(M, prefill2::kBT) * prefill2::kBT;
+    p.o_count = o.count;
+    p.o_rows = o.rows;
+    p.o_vals = o.vals;
+    p.o_cap = (int)o.cap;
+    p.o_extra = partials;   // no K split with outliers: the partial-sum area is free
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(prefill2::kThreads, 1, 1);
     cfg.dynamicSmemBytes = prefill2::kSmemBytes;
@@ -286,7 +314,8 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
         if (d->pairs == 0) {
             cfg.gridDim = dim3((unsigned)d->sms, 1, 1);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, prefill2::prefill2_kernel<false, false>, &cfg) != cudaSuccess ||
+            if (cudaOccupancyMaxActiveClusters(&n, prefill2::prefill2_kernel<false, prefill2::kSym>, &cfg) !=
+                    cudaSuccess ||
                 n < 1) {
                 cudaGetLastError();
                 n = d->sms / 2;
@@ -313,7 +342,7 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
         split_pairs = (int)std::min<int64_t>(P, (int64_t)p.tiles * p.KS);   // at least one K step each
     }
     bool split = false;
-    if (sk_tiles > 0) {
+    if (sk_tiles > 0 && !o.count) {
         const int64_t whole_steps = cdiv(p.tiles, P) * p.KS;
         const int64_t split_steps =
             (int64_t)((p.tiles - sk_tiles) / P) * p.KS + cdiv((int64_t)sk_tiles * p.KS, split_pairs);
@@ -328,13 +357,21 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
         p.sk_iters = 0;
     }
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    using namespace prefill2;
     cudaError_t e;
-    if (zeros)
-        e = split ? cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<true, true>, map, p)
-                  : cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<false, true>, map, p);
-    else
-        e = split ? cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<true, false>, map, p)
-                  : cudaLaunchKernelEx(&cfg, prefill2::prefill2_kernel<false, false>, map, p);
+    if (o.count) {
+        // X^T for the epilogue's outlier term, on the same stream first
+        const dim3 tgrid((unsigned)cdiv(K, 32), (unsigned)(p.Mp / 32), 1);
+        transpose_x_kernel<<<tgrid, dim3(32, 8, 1), 0, st>>>(X, o.xt, (int)M, K, p.Mp);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, prefill2_kernel<false, kOutliers>, map, p);
+    } else if (zeros) {
+        e = split ? cudaLaunchKernelEx(&cfg, prefill2_kernel<true, kZeroPoint>, map, p)
+                  : cudaLaunchKernelEx(&cfg, prefill2_kernel<false, kZeroPoint>, map, p);
+    } else {
+        e = split ? cudaLaunchKernelEx(&cfg, prefill2_kernel<true, kSym>, map, p)
+                  : cudaLaunchKernelEx(&cfg, prefill2_kernel<false, kSym>, map, p);
+    }
     if (e != cudaSuccess) {
         cudaGetLastError();
         return W8_ERR_CUDA;
@@ -391,8 +428,10 @@ static int quantize_common(const void *W, int w_dtype, int64_t K, int64_t N, int
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (percentile > 0.0) {
         if (w_dtype == W8_F32)
-            return launch_percentile<float>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, percentile, q, scales, st);
-        return launch_percentile<__half>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, percentile, q, scales, st);
+            return launch_percentile<float, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, percentile, q,
+                                                   scales, nullptr, nullptr, nullptr, st);
+        return launch_percentile<__half, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, percentile, q,
+                                                scales, nullptr, nullptr, nullptr, st);
     }
     if (asym) {
         if (w_dtype == W8_F32)
@@ -416,6 +455,42 @@ int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, in
 int w8_quantize_per_channel_asym(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
                                  uint16_t *scales, int8_t *zeros, void *stream) {
     return quantize_common(W, w_dtype, K, N, q, scales, zeros, true, stream);
+}
+
+size_t w8_outlier_capacity(int64_t K, double p) {
+    if (K < 1 || !(p > 0.0 && p <= 1.0)) return 0;
+    return (size_t)(K - percentile_rank(K, p));
+}
+
+int w8_quantize_per_channel_outliers(const void *W, int w_dtype, int64_t K, int64_t N, double p, int8_t *q,
+                                     uint16_t *scales, int32_t *o_count, int32_t *o_rows, uint16_t *o_vals,
+                                     void *stream) {
+    if (w_dtype != W8_F32 && w_dtype != W8_F16) return W8_ERR_DTYPE;
+    if (K < 1 || N < 0 || N % 8 != 0 || K > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX * 8 ||
+        !(p > 0.0 && p <= 1.0))
+        return W8_ERR_SHAPE;
+    const int64_t cap = K - percentile_rank(K, p);
+    if (cap > clip::kMaxOutliers) return W8_ERR_LIMIT;
+    if (N == 0) return W8_OK;
+    if (!W || !q || !scales || !o_count || (cap > 0 && (!o_rows || !o_vals))) return W8_ERR_NULL;
+    if (!aligned16(W) || !aligned16(q) || !aligned16(scales)) return W8_ERR_ALIGN;
+    const size_t welem = w_dtype == W8_F32 ? 4 : 2;
+    const size_t wb = (size_t)K * N * welem, qb = (size_t)K * N, cb = (size_t)N * 4,
+                 rb = (size_t)N * cap * 4, vb = (size_t)N * cap * 2;
+    if (overlap(W, wb, q, qb) || overlap(W, wb, scales, (size_t)N * 2) || overlap(q, qb, scales, (size_t)N * 2) ||
+        overlap(o_count, cb, W, wb) || overlap(o_count, cb, q, qb) || overlap(o_rows, rb, W, wb) ||
+        overlap(o_rows, rb, q, qb) || overlap(o_vals, vb, W, wb) || overlap(o_vals, vb, q, qb) ||
+        overlap(o_rows, rb, o_vals, vb) || overlap(o_count, cb, o_rows, rb) || overlap(o_count, cb, o_vals, vb))
+        return W8_ERR_ALIAS;
+    DeviceInfo *d = nullptr;
+    int rc = device_info(&d);
+    if (rc != W8_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (w_dtype == W8_F32)
+        return launch_percentile<float, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, p, q, scales, o_count,
+                                              o_rows, o_vals, st);
+    return launch_percentile<__half, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, p, q, scales, o_count,
+                                           o_rows, o_vals, st);
 }
 
 int w8_quantize_per_channel_clip(const void *W, int w_dtype, int64_t K, int64_t N, int clip_mode,
@@ -496,6 +571,20 @@ static size_t workspace_total(int sms, int64_t N) {
     return partial_area_bytes(sms) + (size_t)cdiv(counters * 4, 256) * 256;
 }
 
+// X^T for the outlier term of the tensor-core path: K rows of M rounded up
+// to the 256-token tile, fp16.
+static size_t xt_bytes(int64_t M, int64_t K) {
+    if (M <= decode::kMaxTokens) return 0;
+    return (size_t)cdiv((int64_t)K * cdiv(M, prefill2::kBT) * prefill2::kBT * 2, 256) * 256;
+}
+
+size_t w8a16_linear_outliers_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+    if (M < 1 || K < 1 || N < 1) return 0;
+    DeviceInfo *d = nullptr;
+    if (device_info(&d) != W8_OK) return 0;
+    return workspace_total(d->sms, N) + xt_bytes(M, K);
+}
+
 size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N) {
     if (M < 1 || K < 1 || N < 1) return 0;
     DeviceInfo *d = nullptr;
@@ -506,7 +595,7 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N) {
 // Both code forms: zeros == nullptr selects the symmetric one.
 static int linear_common(const uint16_t *X, const uint8_t *packed, const uint16_t *scales, const int8_t *zeros,
                          bool asym, const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N,
-                         void *workspace, size_t workspace_bytes, void *stream) {
+                         void *workspace, size_t workspace_bytes, void *stream, Outliers o = Outliers()) {
     if (M < 0 || K < 1 || N < 1 || K % 8 != 0 || N % 8 != 0 || M > (int64_t)INT32_MAX ||
         K > (int64_t)INT32_MAX || cdiv(K, 64) > INT32_MAX)
         return W8_ERR_SHAPE;
@@ -529,8 +618,10 @@ static int linear_common(const uint16_t *X, const uint8_t *packed, const uint16_
     const int KB = (int)cdiv(K, 64);
     const int64_t NB = cdiv(N, 128);
 
-    const size_t need = workspace_total(d->sms, N);
+    const size_t base_need = workspace_total(d->sms, N);
+    const size_t need = o.count ? base_need + xt_bytes(M, K) : base_need;
     if (!workspace || workspace_bytes < need) return W8_ERR_WORKSPACE;
+    if (o.count && M > decode::kMaxTokens) o.xt = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(workspace) + base_need);
     if (overlap(workspace, need, Y, ybytes) || overlap(workspace, need, X, (size_t)M * K * 2))
         return W8_ERR_ALIAS;
     float *partials = static_cast<float *>(workspace);
@@ -550,6 +641,12 @@ static int linear_common(const uint16_t *X, const uint8_t *packed, const uint16_
         p.Y = Y;
         p.partials = partials;
         p.counters = counters;
+        p.X = X;
+        p.K = K;
+        p.o_count = o.count;
+        p.o_rows = o.rows;
+        p.o_vals = o.vals;
+        p.o_cap = (int)o.cap;
         p.M = (int)M;
         p.N = N;
         p.KB = KB;
@@ -574,7 +671,7 @@ static int linear_common(const uint16_t *X, const uint8_t *packed, const uint16_
         }
     }
 
-    return launch_prefill2(d, X, packed, scales, asym ? zeros : nullptr, bias, Y, M, K, N, partials, counters,
+    return launch_prefill2(d, X, packed, scales, asym ? zeros : nullptr, bias, Y, M, K, N, partials, counters, o,
                            st);
 }
 
@@ -583,6 +680,24 @@ int w8a16_linear(const uint16_t *X, const uint8_t *packed, const uint16_t *scale
                  void *workspace, size_t workspace_bytes, void *stream) {
     return linear_common(X, packed, scales, nullptr, false, bias, Y, M, K, N, workspace, workspace_bytes,
                          stream);
+}
+
+int w8a16_linear_outliers(const uint16_t *X, const uint8_t *packed, const uint16_t *scales,
+                          const int32_t *o_count, const int32_t *o_rows, const uint16_t *o_vals, int64_t o_cap,
+                          const uint16_t *bias, uint16_t *Y, int64_t M, int64_t K, int64_t N, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+    if (!o_count || (o_cap > 0 && (!o_rows || !o_vals))) return W8_ERR_NULL;
+    if (o_cap < 0 || o_cap > clip::kMaxOutliers) return W8_ERR_LIMIT;
+    if (M > 0 && Y && (overlap(Y, (size_t)M * N * 2, o_count, (size_t)N * 4) ||
+                       overlap(Y, (size_t)M * N * 2, o_rows, (size_t)N * o_cap * 4) ||
+                       overlap(Y, (size_t)M * N * 2, o_vals, (size_t)N * o_cap * 2)))
+        return W8_ERR_ALIAS;
+    Outliers o;
+    o.count = o_count;
+    o.rows = o_rows;
+    o.vals = o_vals;
+    o.cap = o_cap;
+    return linear_common(X, packed, scales, nullptr, false, bias, Y, M, K, N, workspace, workspace_bytes, stream, o);
 }
 
 int w8a16_linear_asym(const uint16_t *X, const uint8_t *packed, const uint16_t *scales, const int8_t *zeros,
@@ -710,6 +825,12 @@ extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *pack
     p.packed = packed;
     p.scales = scales;
     p.zeros = nullptr;
+    p.X = X;
+    p.K = K;
+    p.o_count = nullptr;
+    p.o_rows = nullptr;
+    p.o_vals = nullptr;
+    p.o_cap = 0;
     p.bias = bias;
     p.Y = Y;
     p.partials = static_cast<float *>(scratch);
