@@ -545,21 +545,32 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                     float ex[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) ex[i] = bb;
-                    for (int j = 0; j < cnt; ++j) {
-                        const int64_t k = p.o_rows[nb * p.o_cap + j];
-                        const float ov = __half2float(__ushort_as_half(p.o_vals[nb * p.o_cap + j]));
-                        const uint4 *src = reinterpret_cast<const uint4 *>(p.XT + k * p.Mp + mb + 32 * cchunk);
+                    // four outliers per round: their X^T rows are loaded
+                    // together (a padding slot reuses a listed row, weight 0)
+                    for (int j0 = 0; j0 < cnt; j0 += 4) {
+                        uint4 xv[4][4];
+                        float ov[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const uint4 xv = src[u];
-                            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int j = j0 + jj < cnt ? j0 + jj : j0;
+                            const int64_t k = p.o_rows[nb * p.o_cap + j];
+                            ov[jj] = j0 + jj < cnt ? __half2float(__ushort_as_half(p.o_vals[nb * p.o_cap + j])) : 0.0f;
+                            const uint4 *src = reinterpret_cast<const uint4 *>(p.XT + k * p.Mp + mb + 32 * cchunk);
 #pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                const __half2 x2 = *reinterpret_cast<const __half2 *>(&xw[h]);
-                                ex[8 * u + 2 * h] = fmaf(__low2float(x2), ov, ex[8 * u + 2 * h]);
-                                ex[8 * u + 2 * h + 1] = fmaf(__high2float(x2), ov, ex[8 * u + 2 * h + 1]);
-                            }
+                            for (int u = 0; u < 4; ++u) xv[jj][u] = src[u];
                         }
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const uint32_t xw[4] = {xv[jj][u].x, xv[jj][u].y, xv[jj][u].z, xv[jj][u].w};
+#pragma unroll
+                                for (int h = 0; h < 4; ++h) {
+                                    const __half2 x2 = *reinterpret_cast<const __half2 *>(&xw[h]);
+                                    ex[8 * u + 2 * h] = fmaf(__low2float(x2), ov[jj], ex[8 * u + 2 * h]);
+                                    ex[8 * u + 2 * h + 1] = fmaf(__high2float(x2), ov[jj], ex[8 * u + 2 * h + 1]);
+                                }
+                            }
                     }
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
@@ -582,33 +593,59 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             const float sc = n_ok ? __half2float(__ushort_as_half(p.scales[n])) : 0.0f;
             const float bi = (n_ok && p.bias) ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
             const int m0 = tb * kBT + 128 * half;
-            if (sg.slot < 0) {
+            if (kMode == kOutliers && sg.slot < 0) {
+                // the parked terms of chunk c + 1 load while chunk c converts;
+                // each chunk is stored right away (no results held)
+                const float4 *xrow = reinterpret_cast<const float4 *>(
+                    p.o_extra + (int64_t)blockIdx.x * kExtraFloats + (threadIdx.x - 256) * 128);
+                float exn[32];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float4 e4 = xrow[u];
+                    exn[4 * u] = e4.x;
+                    exn[4 * u + 1] = e4.y;
+                    exn[4 * u + 2] = e4.z;
+                    exn[4 * u + 3] = e4.w;
+                }
+#pragma unroll
+                for (int cchunk = 0; cchunk < 4; ++cchunk) {
+                    float ex[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ex[i] = exn[i];
+                    if (cchunk < 3) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const float4 e4 = xrow[8 * (cchunk + 1) + u];
+                            exn[4 * u] = e4.x;
+                            exn[4 * u + 1] = e4.y;
+                            exn[4 * u + 2] = e4.z;
+                            exn[4 * u + 3] = e4.w;
+                        }
+                    }
+                    uint32_t v[32];
+                    tmem_load_32(lane_addr + 32 * cchunk, v);
+                    if (cchunk == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_remote(leader(&d_empty));
+                    }
+                    if (n_ok) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int m = m0 + 32 * cchunk + i;
+                            if (m < p.M)
+                                p.Y[(int64_t)m * p.N + n] =
+                                    __half_as_ushort(__float2half_rn(fmaf(__uint_as_float(v[i]), sc, ex[i])));
+                        }
+                    }
+                }
+            } else if (sg.slot < 0) {
                 uint32_t y2[64];
 #pragma unroll
                 for (int cchunk = 0; cchunk < 4; ++cchunk) {
                     uint32_t v[32];
-                    float ex[32];   // outlier form: bias + outlier terms of these tokens
-                    if constexpr (kMode == kOutliers) {
-                        const float4 *srcx = reinterpret_cast<const float4 *>(
-                            p.o_extra + (int64_t)blockIdx.x * kExtraFloats + (threadIdx.x - 256) * 128 + 32 * cchunk);
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const float4 e4 = srcx[u];
-                            ex[4 * u] = e4.x;
-                            ex[4 * u + 1] = e4.y;
-                            ex[4 * u + 2] = e4.z;
-                            ex[4 * u + 3] = e4.w;
-                        }
-                    }
                     tmem_load_32(lane_addr + 32 * cchunk, v);
-                    if constexpr (kMode == kOutliers) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const __half2 hv = __floats2half2_rn(fmaf(__uint_as_float(v[2 * i]), sc, ex[2 * i]),
-                                                                 fmaf(__uint_as_float(v[2 * i + 1]), sc, ex[2 * i + 1]));
-                            y2[16 * cchunk + i] = *reinterpret_cast<const uint32_t *>(&hv);
-                        }
-                    } else {
+                    {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const __half2 hv = __floats2half2_rn(fmaf(__uint_as_float(v[2 * i]), sc, bi),
