@@ -102,6 +102,12 @@ class ClockSampler:
     def mark(self, t0, t1):
         self.windows.append((t0, t1))
 
+    def window_mhz(self, window):
+        """Median SM clock sampled inside one timed window (after stop())."""
+        a, b = window
+        vals = [r[1] for r in getattr(self, "rows", []) if a - 0.15 <= r[0] <= b + 0.15]
+        return statistics.median(vals) if vals else None
+
     def stop(self):
         if self.p is not None:
             self.p.terminate()
@@ -123,6 +129,7 @@ class ClockSampler:
             except Exception:
                 continue
         os.unlink(self.f.name)
+        self.rows = rows
         inside = [r for r in rows if any(a - 0.15 <= r[0] <= b + 0.15 for a, b in self.windows)]
         use = inside if len(inside) >= 2 else rows
         if not use:
@@ -264,6 +271,7 @@ def run_native(args, ws, rank, local):
     torch.cuda.synchronize()
     n_pf = max(5, args.prefill_reps)
     t_pf = timed_replays(g_pf, n_pf, stream, ws, device, sampler)
+    pf_window = sampler.windows[-1]
     pf_s = t_pf / (2 * n_pf)
     pf_flops = 2.0 * M_PREFILL * K_DIM * N_DIM
     pf_tflops = pf_flops / pf_s / 1e12
@@ -303,6 +311,121 @@ def run_native(args, ws, rank, local):
     torch.cuda.synchronize()
     t_e2e = timed_replays(g_e2e, n_rep, stream, ws, device, sampler)
     e2e_value = ws * weight_bytes * steps_done / t_e2e / 1e9
+
+    def graph_time(fn, reps):
+        """Device seconds per call of fn (captured once, replayed)."""
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        g = capture(fn, stream)
+        for _ in range(3):
+            with torch.cuda.stream(stream):
+                g.replay()
+        torch.cuda.synchronize()
+        t = timed_replays(g, reps, stream, ws, device, sampler) / reps
+        del g
+        return t
+
+    # ---- the method's variants on the headline weight (4096 x 27392, 0.1 %
+    # outliers): asymmetric codes, clipped scales, the outlier split
+    variants = {}
+    if not args.no_variants:
+        fl_pf = 2.0 * M_PREFILL * K_DIM * N_DIM
+        qa, sa, za = w8.quantize_asym(W)
+        pa = [w8.prepack(qa) for _ in range(2)]
+        t_qa = graph_time(lambda: w8.quantize_asym(W, qa, sa, za), 20)
+        t_da = graph_time(lambda: [w8.linear_asym(X1, c, sa, za, out=Y1, workspace=work) for c in pa], 200) / 2
+        t_pa = graph_time(lambda: [w8.linear_asym(Xp, c, sa, za, out=Yp) for c in pa], 20) / 2
+        variants["asymmetric"] = {
+            "quantize_us": round(t_qa * 1e6, 1), "quantize_GBps": round(q_bytes / t_qa / 1e9, 1),
+            "decode_m1_us": round(t_da * 1e6, 2), "decode_m1_weight_GBps": round(weight_bytes / t_da / 1e9, 1),
+            "decode_m1_frac_hbm": round(alg_bytes / t_da / 1e9 / hbm_peak, 4),
+            "prefill_m2048_us": round(t_pa * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_pa / 1e12, 1)}
+        del pa
+        qc = torch.empty_like(q)
+        sc_ = torch.empty_like(scales)
+        t_cf = graph_time(lambda: w8.quantize_clip(W, "fixed", 0.05, qc, sc_), 20)
+        t_cp = graph_time(lambda: w8.quantize_clip(W, "percentile", 0.999, qc, sc_), 5)
+        variants["clip_fixed"] = {"clip": 0.05, "quantize_us": round(t_cf * 1e6, 1),
+                                  "quantize_GBps": round(q_bytes / t_cf / 1e9, 1)}
+        variants["clip_percentile"] = {"p": 0.999, "quantize_us": round(t_cp * 1e6, 1),
+                                       "quantize_GBps": round(q_bytes / t_cp / 1e9, 1),
+                                       "passes_over_W": 5}
+        qo, so, co, ro, vo = w8.quantize_outliers(W, 0.999)
+        po = [w8.prepack(qo) for _ in range(2)]
+        t_qo = graph_time(lambda: w8.quantize_outliers(W, 0.999), 5)
+        t_do = graph_time(lambda: [w8.linear_outliers(X1, c, so, co, ro, vo, out=Y1) for c in po], 200) / 2
+        t_po = graph_time(lambda: [w8.linear_outliers(Xp, c, so, co, ro, vo, out=Yp) for c in po], 20) / 2
+        variants["outlier_split"] = {
+            "p": 0.999, "outliers_per_channel": int(ro.shape[1]), "quantize_us": round(t_qo * 1e6, 1),
+            "decode_m1_us": round(t_do * 1e6, 2), "decode_m1_weight_GBps": round(weight_bytes / t_do / 1e9, 1),
+            "prefill_m2048_us": round(t_po * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_po / 1e12, 1)}
+        del po, qo, qc
+        torch.cuda.empty_cache()
+
+    # ---- the prefill sweep: M in {512, 1024, 2048} on 4096 x 27392 and
+    # 13696 x 4096 (the latter's few tiles take the K split at M = 512)
+    prefill_sweep = {}
+    if not args.no_variants:
+        sw = synthetic.WORKLOADS["chatglm2_prefill"]
+        for i, (Ks, Ns) in enumerate(sw["matrices"]):
+            Ws = torch.from_numpy(synthetic.weights(Ks, Ns, seed, synthetic.tensor_id(4, 0, i, 0),
+                                                    outlier_frac=0.001)).to(device)
+            qs, ss = w8.quantize(Ws)
+            del Ws
+            ncp = 2 if Ks * Ns > 64 << 20 else 4
+            ps = [w8.prepack(qs) for _ in range(ncp)]
+            row = {}
+            for Ms in sw["M"]:
+                Xs = torch.from_numpy(synthetic.activations(Ms, Ks, seed, synthetic.tensor_id(4, Ms, i, 1))).to(device)
+                Ysw = torch.empty((Ms, Ns), dtype=torch.float16, device=device)
+                t = graph_time(lambda: [w8.linear(Xs, c, ss, out=Ysw) for c in ps], 20) / ncp
+                tf = 2.0 * Ms * Ks * Ns / t / 1e12
+                row[f"M={Ms}"] = {"us": round(t * 1e6, 1), "TFLOPs": round(tf, 1),
+                                  "frac_tensor_sustained": round(tf / tf_sustained, 4)}
+                del Xs, Ysw
+            prefill_sweep[f"{Ks}x{Ns}"] = row
+            del ps, qs
+        torch.cuda.empty_cache()
+
+    # ---- BERT-base, 4096 tokens: quantize all 12 layers' 48 weights, then
+    # the four linears of a layer at M = 4096 (distinct weights per layer)
+    bert = {}
+    if not args.no_variants:
+        bw = synthetic.WORKLOADS["bert_base_4096_tokens"]
+        Wb, qb, sb, pb = [], [], [], []
+        for i, (Kb, Nb) in enumerate(bw["matrices"]):
+            w0 = torch.from_numpy(synthetic.weights(Kb, Nb, seed, synthetic.tensor_id(5, 0, i, 0))).to(device)
+            Wb.append([w0] + [w0.clone() for _ in range(bw["layers"] - 1)])
+            qb.append([torch.empty((Kb, Nb), dtype=torch.int8, device=device) for _ in range(bw["layers"])])
+            sb.append([torch.empty((Nb,), dtype=torch.float16, device=device) for _ in range(bw["layers"])])
+        def bert_quantize():
+            for i in range(len(Wb)):
+                for l in range(bw["layers"]):
+                    w8.quantize(Wb[i][l], qb[i][l], sb[i][l])
+        t_bq = graph_time(bert_quantize, 5)
+        bq_bytes = bw["layers"] * sum(Kb * Nb * 5 + 2 * Nb for Kb, Nb in bw["matrices"])
+        for i in range(len(Wb)):
+            pb.append([w8.prepack(qb[i][l]) for l in range(bw["layers"])])
+        del Wb
+        Mb = bw["M"][0]
+        Xb = [torch.from_numpy(synthetic.activations(Mb, Kb, seed, synthetic.tensor_id(5, 0, i, 1))).to(device)
+              for i, (Kb, Nb) in enumerate(bw["matrices"])]
+        Yb = [torch.empty((Mb, Nb), dtype=torch.float16, device=device) for Kb, Nb in bw["matrices"]]
+        def bert_layers():
+            for l in range(bw["layers"]):
+                for i in range(len(pb)):
+                    w8.linear(Xb[i], pb[i][l], sb[i][l], out=Yb[i])
+        t_bl = graph_time(bert_layers, 5)
+        bl_flops = bw["layers"] * sum(2.0 * Mb * Kb * Nb for Kb, Nb in bw["matrices"])
+        bert = {"workload": "BERT-base, 4096 tokens: QKV 768x2304, out 768x768, FFN 768x3072 and 3072x768, "
+                            "x 12 layers (distinct weights)",
+                "quantize_all_us": round(t_bq * 1e6, 1), "quantize_GBps": round(bq_bytes / t_bq / 1e9, 1),
+                "quantize_launches": len(bw["matrices"]) * bw["layers"],
+                "linears_us_per_layer": round(t_bl * 1e6 / bw["layers"], 1),
+                "linears_TFLOPs": round(bl_flops / t_bl / 1e12, 1)}
+        del pb, Xb, Yb, qb
+        torch.cuda.empty_cache()
 
     # ---- the ChatGLM2-6B decode layer set: 28 layers x 4 linears (QKV,
     # dense, h-to-4h, 4h-to-h), each call on its own weight buffer (5.7 GB
@@ -357,6 +480,7 @@ def run_native(args, ws, rank, local):
         del packed_set
 
     clocks = sampler.stop()
+    pf_mhz = sampler.window_mhz(pf_window)
 
     out = {
         "metric": METRIC,
@@ -390,6 +514,8 @@ def run_native(args, ws, rank, local):
         "prefill": {
             "metric": "TFLOP/s (M=2048, 4096x27392)", "value": round(pf_tflops, 1), "unit": "TFLOP/s",
             "us_per_call": round(pf_s * 1e6, 2),
+            "calls_timed": 2 * n_pf,
+            "sm_mhz_median_in_region": pf_mhz,
             # the prefill timed region is a long back-to-back loop under the
             # power cap, the condition of the sustained GEMM measurement
             "roofline": {"bound": "tensor", "achieved": round(pf_tflops, 1), "peak": tf_sustained,
@@ -415,6 +541,9 @@ def run_native(args, ws, rank, local):
         "decode_set": ({"workload": "ChatGLM2-6B decode linears, 28 layers x (QKV 4096x4608, dense 4096x4096, "
                                     "h-to-4h 4096x27392, 4h-to-h 13696x4096), distinct weight buffers, one CUDA graph",
                         **decode_set} if decode_set else None),
+        "variants": variants or None,
+        "prefill_sweep": prefill_sweep or None,
+        "bert_base_4096": bert or None,
         "gpu_launches": steps_done,
         "clocks": clocks,
     }
@@ -528,6 +657,8 @@ def main():
     ap.add_argument("--no-decode-set", action="store_true",
                     help="skip the 28-layer decode set measurement")
     ap.add_argument("--set-reps", type=int, default=100)
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the variant, prefill-sweep and BERT sections")
     ap.add_argument("--profile", choices=["decode", "decode16", "prefill", "quantize", "prepack"],
                     help="run --steps plain launches of one kernel (for ncu) and exit")
     args = ap.parse_args()
