@@ -490,8 +490,6 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                             c[t][i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&w_empty[wr.s]);
                 if (!warp_all(mbar_wait(&a_empty[ar.s], ar.ph ^ 1u, SITE_P2_AEMPTY))) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
@@ -511,11 +509,14 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                             }
                         }
                     }
-                    tmem_st_32x32b_x32(lane_addr + kAcol0 + 32 * kKStep * ar.s + 32 * t, v);
+                    tmem_store_32(lane_addr + kAcol0 + 32 * kKStep * ar.s + 32 * t, v);
                 }
-                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
+                // the slot is released only now that every lane's codes are
+                // used: released right after the shared loads were issued, a
+                // load still in flight could see the next bulk copy's bytes
+                if (lane == 0) mbar_arrive(&w_empty[wr.s]);
                 if (lane == 0) mbar_arrive_remote(leader(&a_full[ar.s]));
                 wr.next(kWStages);
                 ar.next(kABuf);

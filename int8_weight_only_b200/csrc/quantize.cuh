@@ -284,6 +284,14 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                             for (int e = 0; e < B::kCols; ++e) amax[e] = fmaxf(amax[e], fabsf(v[e]));
                         }
                     }
+                    // the slot's values are in registers before it is released
+                    // (arithmetic alone could be scheduled after the arrive,
+                    // with a load still reading the slot the next copy fills)
+#pragma unroll
+                    for (int e = 0; e < B::kCols; ++e) {
+                        asm volatile("" ::"f"(amax[e]));
+                        if constexpr (kAsym) asm volatile("" ::"f"(amin[e]));
+                    }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
                     if (++s == kStages) { s = 0; ph ^= 1u; }
