@@ -399,11 +399,19 @@ def run_native(args, ws, rank, local):
             Wb.append([w0] + [w0.clone() for _ in range(bw["layers"] - 1)])
             qb.append([torch.empty((Kb, Nb), dtype=torch.int8, device=device) for _ in range(bw["layers"])])
             sb.append([torch.empty((Nb,), dtype=torch.float16, device=device) for _ in range(bw["layers"])])
-        def bert_quantize():
-            for i in range(len(Wb)):
-                for l in range(bw["layers"]):
-                    w8.quantize(Wb[i][l], qb[i][l], sb[i][l])
-        t_bq = graph_time(bert_quantize, 5)
+        flat_w = [Wb[i][l] for i in range(len(Wb)) for l in range(bw["layers"])]
+        flat_q = [qb[i][l] for i in range(len(Wb)) for l in range(bw["layers"])]
+        flat_s = [sb[i][l] for i in range(len(Wb)) for l in range(bw["layers"])]
+
+        def bert_quantize_each():
+            for W_, q_, s_ in zip(flat_w, flat_q, flat_s):
+                w8.quantize(W_, q_, s_)
+
+        def bert_quantize_batched():
+            w8.quantize_batched(flat_w, flat_q, flat_s)
+
+        t_bq1 = graph_time(bert_quantize_each, 5)
+        t_bq = graph_time(bert_quantize_batched, 5)
         bq_bytes = bw["layers"] * sum(Kb * Nb * 5 + 2 * Nb for Kb, Nb in bw["matrices"])
         for i in range(len(Wb)):
             pb.append([w8.prepack(qb[i][l]) for l in range(bw["layers"])])
@@ -421,7 +429,8 @@ def run_native(args, ws, rank, local):
         bert = {"workload": "BERT-base, 4096 tokens: QKV 768x2304, out 768x768, FFN 768x3072 and 3072x768, "
                             "x 12 layers (distinct weights)",
                 "quantize_all_us": round(t_bq * 1e6, 1), "quantize_GBps": round(bq_bytes / t_bq / 1e9, 1),
-                "quantize_launches": len(bw["matrices"]) * bw["layers"],
+                "quantize_launches": 1,
+                "quantize_one_launch_per_weight_us": round(t_bq1 * 1e6, 1),
                 "linears_us_per_layer": round(t_bl * 1e6 / bw["layers"], 1),
                 "linears_TFLOPs": round(bl_flops / t_bl / 1e12, 1)}
         del pb, Xb, Yb, qb

@@ -107,6 +107,20 @@ int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N,
  * Other arguments, exactness and errors as w8_quantize_per_channel (zeros
  * must not overlap W, q or scales).
  */
+/*
+ * w8_quantize_per_channel_batched -- w8_quantize_per_channel for `count`
+ * weights in as few launches as possible (up to 64 weights per launch: the
+ * launch's clusters walk all their column panels), e.g. every weight of a
+ * model at load time (BERT-base: 48).  The arrays are host arrays of
+ * length count: W[i] [K[i], N[i]] (all of dtype w_dtype), q[i] [K[i], N[i]]
+ * int8 and scales[i] [N[i]] fp16 device pointers.  The result equals
+ * `count` separate w8_quantize_per_channel calls bit for bit.  No output
+ * may overlap any weight or any other output.  count == 0 and entries with
+ * N[i] == 0 are no-ops.  Errors as w8_quantize_per_channel.
+ */
+int w8_quantize_per_channel_batched(int count, const void *const *W, int w_dtype, const int64_t *K,
+                                    const int64_t *N, int8_t *const *q, uint16_t *const *scales, void *stream);
+
 int w8_quantize_per_channel_asym(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
                                  uint16_t *scales, int8_t *zeros, void *stream);
 

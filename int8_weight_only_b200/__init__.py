@@ -18,7 +18,7 @@ import os
 import threading
 
 __all__ = [
-    "W8Error", "load_library", "library_path", "quantize", "quantize_asym", "quantize_clip", "quantize_outliers", "prepack", "unpack",
+    "W8Error", "load_library", "library_path", "quantize", "quantize_batched", "quantize_asym", "quantize_clip", "quantize_outliers", "prepack", "unpack",
     "prepacked_bytes", "workspace_bytes", "linear", "linear_asym", "linear_outliers", "linear_decode_static", "W8A16Linear", "device_status",
     "test_bounded_wait", "STATUS",
 ]
@@ -62,6 +62,7 @@ def load_library():
         vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
         lib.w8_quantize_per_channel.argtypes = [vp, i32, i64, i64, vp, vp, vp]
         lib.w8_quantize_per_channel_asym.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
+        lib.w8_quantize_per_channel_batched.argtypes = [i32, vp, i32, vp, vp, vp, vp, vp]
         lib.w8_quantize_per_channel_clip.argtypes = [vp, i32, i64, i64, i32, ctypes.c_double, vp, vp, vp]
         lib.w8_outlier_capacity.argtypes = [i64, ctypes.c_double]
         lib.w8_outlier_capacity.restype = sz
@@ -147,6 +148,43 @@ def quantize(W, q=None, scales=None):
         _check(lib.w8_quantize_per_channel(_ptr(W), dt, K, N, _ptr(q), _ptr(scales), _stream(W.device)),
                "w8_quantize_per_channel")
     return q, scales
+
+
+def quantize_batched(Ws, qs=None, scales=None):
+    """Per-output-channel symmetric int8 quantization of several weights in
+    as few launches as possible (up to 64 per launch).  Ws: list of [K, N]
+    tensors of one dtype (float32 or float16) on one device.  Returns
+    (list of q int8, list of scales fp16), bit for bit those of quantize."""
+    torch = _torch()
+    lib = load_library()
+    Ws = list(Ws)
+    if not Ws:
+        return [], []
+    dev = Ws[0].device
+    dtype = Ws[0].dtype
+    for W in Ws:
+        _need_cuda(W, "W")
+        if W.dim() != 2 or W.dtype != dtype or W.device != dev:
+            raise ValueError("Ws must be 2-D tensors of one dtype on one device")
+    if dtype == torch.float32:
+        dt = W8_F32
+    elif dtype == torch.float16:
+        dt = W8_F16
+    else:
+        raise ValueError("W must be float32 or float16")
+    if qs is None:
+        qs = [torch.empty(tuple(W.shape), dtype=torch.int8, device=dev) for W in Ws]
+    if scales is None:
+        scales = [torch.empty((W.shape[1],), dtype=torch.float16, device=dev) for W in Ws]
+    n = len(Ws)
+    arr_p = ctypes.c_void_p * n
+    arr_i = ctypes.c_int64 * n
+    with torch.cuda.device(dev):
+        _check(lib.w8_quantize_per_channel_batched(
+            n, arr_p(*[W.data_ptr() for W in Ws]), dt, arr_i(*[W.shape[0] for W in Ws]),
+            arr_i(*[W.shape[1] for W in Ws]), arr_p(*[q.data_ptr() for q in qs]),
+            arr_p(*[s.data_ptr() for s in scales]), _stream(dev)), "w8_quantize_per_channel_batched")
+    return qs, scales
 
 
 def quantize_asym(W, q=None, scales=None, zeros=None):

@@ -137,17 +137,55 @@ __device__ __forceinline__ void load_seg<__half>(const uint8_t *p, float (&v)[8]
     }
 }
 
-struct Params {
+// A launch quantizes a batch of up to kMaxBatch weights (one weight is a
+// batch of one): the clusters walk one global panel index over all of
+// them, and each panel finds its weight in the table.
+constexpr int kMaxBatch = 64;
+
+struct Mat {
     int8_t *q;
     uint16_t *scales;
     int8_t *zeros;     // asymmetric form only: [N] zero points
-    float clip;        // symmetric form: bound = min(max|W|, clip); +inf: no clip
     int64_t K;
     int64_t N;
     int kc;            // rows per cluster rank (multiple of the box height)
-    int panels;        // ceil(N / 32)
-    int clusters;      // clusters in the grid
+    int panel0;        // this weight's first global panel
 };
+
+// kCap: the table's capacity (1 for a single weight, whose lookups then
+// fold away; kMaxBatch for a batch).
+template <int kCap>
+struct Params {
+    CUtensorMap maps[kCap];   // per weight: W [K, N], box 32 columns x Box<T>::kRows rows
+    Mat mats[kCap];
+    int count;
+    int panels;        // all weights' panels, ceil(N / 32) each
+    int clusters;      // clusters in the grid
+    float clip;        // symmetric form: bound = min(max|W|, clip); +inf: no clip
+};
+
+// Global panel g: its weight, its panel within the weight, and this
+// cluster rank's rows of it.
+struct PanelRef {
+    int m;
+    int local;
+    int64_t k_begin, k_end;
+    int nbox;
+};
+
+template <int kRows, int kCap>
+__device__ __forceinline__ PanelRef panel_ref(const Params<kCap> &p, int g, uint32_t rank) {
+    int m = 0;
+    if constexpr (kCap > 1)
+        while (m + 1 < p.count && p.mats[m + 1].panel0 <= g) ++m;
+    PanelRef r;
+    r.m = m;
+    r.local = g - p.mats[m].panel0;
+    r.k_begin = (int64_t)rank * p.mats[m].kc;
+    r.k_end = min64(p.mats[m].K, r.k_begin + p.mats[m].kc);
+    r.nbox = (int)((max64(0, r.k_end - r.k_begin) + kRows - 1) / kRows);
+    return r;
+}
 
 // grid = clusters * C CTAs, cluster dims (C, 1, 1), kThreads threads,
 // kSmemBytes dynamic shared memory.  The tensor map covers W [K, N] with
@@ -168,9 +206,9 @@ struct Params {
 // kAsym: the asymmetric form -- pass 1 keeps the column minimum and maximum
 // (both start at 0: the range always holds 0), the exchange combines both,
 // and pass 2 writes clamp(rne(w / s) + z, -128, 127).
-template <typename T, bool kAsym>
+template <typename T, bool kAsym, int kCap>
 __global__ void __launch_bounds__(kThreads, 2)
-quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
+quantize_kernel(const __grid_constant__ Params<kCap> p) {
     using B = Box<T>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *ring = reinterpret_cast<uint8_t *>(
@@ -192,10 +230,6 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
     const uint32_t rank = cluster_rank();
     const uint32_t csize = cluster_size();
     const int cid = blockIdx.x / csize;
-    const int64_t k_begin = (int64_t)rank * p.kc;
-    const int64_t k_end = min64(p.K, k_begin + p.kc);
-    const int rows = (int)max64(0, k_end - k_begin);
-    const int nbox = (rows + B::kRows - 1) / B::kRows;
     const int npan = cid < p.panels ? (p.panels - cid + p.clusters - 1) / p.clusters : 0;
 
     if (threadIdx.x == 0) {
@@ -207,7 +241,7 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
         mbar_init(&xbar[1], csize);
         mbar_init(&cbar, kConsumers);
         fence_barrier_init();
-        prefetch_tensormap(&tmap_w);
+        if (cid < p.panels) prefetch_tensormap(&p.maps[panel_ref<B::kRows, kCap>(p, cid, rank).m]);
     }
     // barrier initialisation is visible to the whole cluster before any
     // remote arrive
@@ -226,12 +260,12 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                     // pass 0: P1 of panel j; pass 1: P2 of panel j - 1
                     const int pj = pass == 0 ? j : j - 1;
                     if (pj < 0 || pj >= npan) continue;
-                    const int panel = cid + pj * p.clusters;
-                    for (int i = 0; i < nbox; ++i) {
+                    const PanelRef pr = panel_ref<B::kRows, kCap>(p, cid + pj * p.clusters, rank);
+                    for (int i = 0; i < pr.nbox; ++i) {
                         if (!mbar_wait_parked(&empty[s], ph ^ 1u, SITE_Q_EMPTY)) { ok = false; break; }
                         mbar_arrive_expect_tx(&full[s], kBoxBytes);
-                        tma_load_2d_hint(ring + s * kBoxBytes, &tmap_w, panel * kPanel,
-                                         (int32_t)(k_begin + (int64_t)i * B::kRows), &full[s],
+                        tma_load_2d_hint(ring + s * kBoxBytes, &p.maps[pr.m], pr.local * kPanel,
+                                         (int32_t)(pr.k_begin + (int64_t)i * B::kRows), &full[s],
                                          pass == 0 ? keep : drop);
                         ++issued;
                         if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -263,10 +297,11 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
         for (int j = 0; j <= npan && ok; ++j) {
             // ---------------- (a) pass 1 over panel j: column |max|
             if (j < npan) {
+                const PanelRef pr1 = panel_ref<B::kRows, kCap>(p, cid + j * p.clusters, rank);
                 float amax[B::kCols], amin[B::kCols];   // amin: asymmetric form only
 #pragma unroll
                 for (int e = 0; e < B::kCols; ++e) amax[e] = amin[e] = 0.0f;
-                for (int i = 0; i < nbox; ++i) {
+                for (int i = 0; i < pr1.nbox; ++i) {
                     if (!warp_all(mbar_wait_parked(&full[s], ph, SITE_Q_LOAD))) { ok = false; break; }
                     const uint8_t *box = ring + s * kBoxBytes;
 #pragma unroll
@@ -334,7 +369,12 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
             }
             // ---------------- (b) combine the maxima of panel j - 1
             const int pj = j - 1;
-            const int panel = cid + pj * p.clusters;
+            const PanelRef pr = panel_ref<B::kRows, kCap>(p, cid + pj * p.clusters, rank);
+            // this weight's outputs, read from the parameter table once
+            const int64_t mN = p.mats[pr.m].N;
+            int8_t *const mq = p.mats[pr.m].q;
+            uint16_t *const ms = p.mats[pr.m].scales;
+            int8_t *const mz = p.mats[pr.m].zeros;
             if (!warp_all(mbar_wait_cluster(&xbar[pj & 1], (pj >> 1) & 1, SITE_Q_XCHG))) { ok = false; break; }
             if (c < kPanel) {
                 float m = 0.0f;
@@ -354,10 +394,10 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                 col_scale[c] = sf;
                 col_inv[c] = sf != 0.0f ? __frcp_rn(sf) : 0.0f;
                 col_zero[c] = z;
-                const int64_t n = (int64_t)panel * kPanel + c;
-                if (rank == 0 && n < p.N) {
-                    p.scales[n] = __half_as_ushort(s16);
-                    if constexpr (kAsym) p.zeros[n] = (int8_t)z;
+                const int64_t n = (int64_t)pr.local * kPanel + c;
+                if (rank == 0 && n < mN) {
+                    ms[n] = __half_as_ushort(s16);
+                    if constexpr (kAsym) mz[n] = (int8_t)z;
                 }
             }
             // every consumer's partial maxima of panel j are in part[] and
@@ -375,9 +415,9 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                 inv[e] = col_inv[col0 + e];
                 zp[e] = col_zero[col0 + e];
             }
-            const int64_t n0 = (int64_t)panel * kPanel + col0;
-            const bool cols_ok = n0 < p.N;   // N % 8 == 0: a segment is all in or all out
-            for (int i = 0; i < nbox; ++i) {
+            const int64_t n0 = (int64_t)pr.local * kPanel + col0;
+            const bool cols_ok = n0 < mN;   // N % 8 == 0: a segment is all in or all out
+            for (int i = 0; i < pr.nbox; ++i) {
                 if (!warp_all(mbar_wait_parked(&full[s], ph, SITE_Q_LOAD))) { ok = false; break; }
                 const uint8_t *box = ring + s * kBoxBytes;
 #pragma unroll
@@ -413,9 +453,9 @@ quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Params p) {
                         const uint32_t hi = __byte_perm((uint32_t)code[4 * g + 2], (uint32_t)code[4 * g + 3], 0x0040);
                         packed[g] = __byte_perm(lo, hi, 0x5410);
                     }
-                    const int64_t k = k_begin + (int64_t)i * B::kRows + rloc;
-                    if (k < k_end && cols_ok) {
-                        int8_t *dst = p.q + k * p.N + n0;
+                    const int64_t k = pr.k_begin + (int64_t)i * B::kRows + rloc;
+                    if (k < pr.k_end && cols_ok) {
+                        int8_t *dst = mq + k * mN + n0;
                         if (B::kCols == 4)
                             *reinterpret_cast<uint32_t *>(dst) = packed[0];
                         else

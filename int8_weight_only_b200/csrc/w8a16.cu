@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstring>
 #include <climits>
 #include <mutex>
 
@@ -71,10 +72,12 @@ int device_info(DeviceInfo **out) {
             smem((const void *)prefill2::prefill2_kernel<false, prefill2::kZeroPoint>, prefill2::kSmemBytes);
             smem((const void *)prefill2::prefill2_kernel<true, prefill2::kZeroPoint>, prefill2::kSmemBytes);
             smem((const void *)prefill2::prefill2_kernel<false, prefill2::kOutliers>, prefill2::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<float, false>, quant::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<__half, false>, quant::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<float, true>, quant::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<__half, true>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<float, false, 1>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<__half, false, 1>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<float, true, 1>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<__half, true, 1>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<float, false, quant::kMaxBatch>, quant::kSmemBytes);
+            smem((const void *)quant::quantize_kernel<__half, false, quant::kMaxBatch>, quant::kSmemBytes);
             smem((const void *)clip::percentile_quantize_kernel<float, false>, clip::kSmemBytes);
             smem((const void *)clip::percentile_quantize_kernel<__half, false>, clip::kSmemBytes);
             smem((const void *)clip::percentile_quantize_kernel<float, true>, clip::kSmemBytes);
@@ -139,19 +142,40 @@ inline int quantize_cluster(int64_t K, int rows_per_box) {
     return (int)std::max<int64_t>(1, std::min<int64_t>(4, cdiv(K, 2 * rows_per_box)));
 }
 
-template <typename T, bool kAsym>
-int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_t K, int64_t N,
-                    int8_t *q, uint16_t *scales, int8_t *zeros, float clip_bound, cudaStream_t st) {
+// A batch of up to quant::kMaxBatch weights in one launch (one weight is a
+// batch of one).  The cluster size follows the largest K.
+template <typename T, bool kAsym, int kCap>
+int launch_quantize(DeviceInfo *d, int count, const void *const *W, CUtensorMapDataType dt, const int64_t *K,
+                    const int64_t *N, int8_t *const *q, uint16_t *const *scales, int8_t *const *zeros,
+                    float clip_bound, cudaStream_t st) {
     constexpr int rows = quant::Box<T>::kRows;
-    const int C = quantize_cluster(K, rows);
-    const int64_t kc = cdiv(cdiv(K, C), rows) * rows;
-    const int64_t panels = cdiv(N, quant::kPanel);
-    if (kc > INT32_MAX || panels > INT32_MAX) return W8_ERR_SHAPE;
-
-    CUtensorMap map;
-    int rc = make_map_2d(&map, W, dt, (int)sizeof(T), (uint64_t)N, (uint64_t)K, quant::kPanel, rows,
-                         CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (rc != W8_OK) return rc;
+    int64_t kmax = 1;
+    for (int i = 0; i < count; ++i) kmax = std::max(kmax, K[i]);
+    const int C = quantize_cluster(kmax, rows);
+    static thread_local quant::Params<kCap> p;   // up to about 12 KB: not on the stack
+    if (count > kCap) return W8_ERR_SHAPE;
+    memset(&p, 0, sizeof(p));
+    int64_t panels = 0;
+    for (int i = 0; i < count; ++i) {
+        const int64_t kc = cdiv(cdiv(K[i], C), rows) * rows;
+        if (kc > INT32_MAX) return W8_ERR_SHAPE;
+        int rc = make_map_2d(&p.maps[i], W[i], dt, (int)sizeof(T), (uint64_t)N[i], (uint64_t)K[i], quant::kPanel,
+                             rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (rc != W8_OK) return rc;
+        p.mats[i].q = q[i];
+        p.mats[i].scales = scales[i];
+        p.mats[i].zeros = zeros ? zeros[i] : nullptr;
+        p.mats[i].K = K[i];
+        p.mats[i].N = N[i];
+        p.mats[i].kc = (int)kc;
+        p.mats[i].panel0 = (int)panels;
+        panels += cdiv(N[i], quant::kPanel);
+        if (panels > INT32_MAX) return W8_ERR_SHAPE;
+    }
+    p.count = count;
+    p.panels = (int)panels;
+    p.clip = clip_bound;
+    if (panels == 0) return W8_OK;
 
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(quant::kThreads, 1, 1);
@@ -173,7 +197,7 @@ int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_
         if (cached == 0) {
             cfg.gridDim = dim3((unsigned)(C * d->sms), 1, 1);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, quant::quantize_kernel<T, kAsym>, &cfg) != cudaSuccess ||
+            if (cudaOccupancyMaxActiveClusters(&n, quant::quantize_kernel<T, kAsym, kCap>, &cfg) != cudaSuccess ||
                 n < 1) {
                 cudaGetLastError();
                 n = std::max(1, d->sms / C);
@@ -182,18 +206,9 @@ int launch_quantize(DeviceInfo *d, const void *W, CUtensorMapDataType dt, int64_
         }
         resident = cached;
     }
-    quant::Params p;
-    p.q = q;
-    p.scales = scales;
-    p.zeros = zeros;
-    p.clip = clip_bound;
-    p.K = K;
-    p.N = N;
-    p.kc = (int)kc;
-    p.panels = (int)panels;
     p.clusters = (int)std::min<int64_t>(panels, resident);
     cfg.gridDim = dim3((unsigned)(p.clusters * C), 1, 1);
-    if (cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T, kAsym>, map, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T, kAsym, kCap>, p) != cudaSuccess) {
         cudaGetLastError();
         return W8_ERR_CUDA;
     }
@@ -435,16 +450,16 @@ static int quantize_common(const void *W, int w_dtype, int64_t K, int64_t N, int
     }
     if (asym) {
         if (w_dtype == W8_F32)
-            return launch_quantize<float, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, zeros,
-                                                INFINITY, st);
-        return launch_quantize<__half, true>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, zeros,
-                                             INFINITY, st);
+            return launch_quantize<float, true, 1>(d, 1, &W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, &K, &N, &q, &scales,
+                                                &zeros, INFINITY, st);
+        return launch_quantize<__half, true, 1>(d, 1, &W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, &K, &N, &q, &scales,
+                                             &zeros, INFINITY, st);
     }
     if (w_dtype == W8_F32)
-        return launch_quantize<float, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, K, N, q, scales, nullptr,
-                                             clip_bound, st);
-    return launch_quantize<__half, false>(d, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, K, N, q, scales, nullptr,
-                                          clip_bound, st);
+        return launch_quantize<float, false, 1>(d, 1, &W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, &K, &N, &q, &scales,
+                                             nullptr, clip_bound, st);
+    return launch_quantize<__half, false, 1>(d, 1, &W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, &K, &N, &q, &scales,
+                                          nullptr, clip_bound, st);
 }
 
 int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
@@ -455,6 +470,66 @@ int w8_quantize_per_channel(const void *W, int w_dtype, int64_t K, int64_t N, in
 int w8_quantize_per_channel_asym(const void *W, int w_dtype, int64_t K, int64_t N, int8_t *q,
                                  uint16_t *scales, int8_t *zeros, void *stream) {
     return quantize_common(W, w_dtype, K, N, q, scales, zeros, true, stream);
+}
+
+int w8_quantize_per_channel_batched(int count, const void *const *W, int w_dtype, const int64_t *K,
+                                    const int64_t *N, int8_t *const *q, uint16_t *const *scales, void *stream) {
+    if (count < 0) return W8_ERR_SHAPE;
+    if (count == 0) return W8_OK;
+    if (!W || !K || !N || !q || !scales) return W8_ERR_NULL;
+    if (w_dtype != W8_F32 && w_dtype != W8_F16) return W8_ERR_DTYPE;
+    const size_t welem = w_dtype == W8_F32 ? 4 : 2;
+    for (int i = 0; i < count; ++i) {
+        if (K[i] < 1 || N[i] < 0 || N[i] % 8 != 0 || K[i] > (int64_t)INT32_MAX || N[i] > (int64_t)INT32_MAX * 8)
+            return W8_ERR_SHAPE;
+        if (N[i] == 0) continue;
+        if (!W[i] || !q[i] || !scales[i]) return W8_ERR_NULL;
+        if (!aligned16(W[i]) || !aligned16(q[i]) || !aligned16(scales[i])) return W8_ERR_ALIGN;
+    }
+    // no output overlaps any weight or any other output
+    for (int i = 0; i < count; ++i) {
+        if (N[i] == 0) continue;
+        const size_t qb = (size_t)K[i] * N[i], sb = (size_t)N[i] * 2;
+        if (overlap(q[i], qb, scales[i], sb)) return W8_ERR_ALIAS;
+        for (int j = 0; j < count; ++j) {
+            if (N[j] == 0) continue;
+            const size_t wb = (size_t)K[j] * N[j] * welem;
+            if (overlap(q[i], qb, W[j], wb) || overlap(scales[i], sb, W[j], wb)) return W8_ERR_ALIAS;
+            if (j != i && (overlap(q[i], qb, q[j], (size_t)K[j] * N[j]) ||
+                           overlap(scales[i], sb, scales[j], (size_t)N[j] * 2) ||
+                           overlap(q[i], qb, scales[j], (size_t)N[j] * 2)))
+                return W8_ERR_ALIAS;
+        }
+    }
+    DeviceInfo *d = nullptr;
+    int rc = device_info(&d);
+    if (rc != W8_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int i0 = 0; i0 < count; i0 += quant::kMaxBatch) {
+        // the weights with N > 0 of this chunk, in order
+        const void *w[quant::kMaxBatch];
+        int64_t k[quant::kMaxBatch], n[quant::kMaxBatch];
+        int8_t *qq[quant::kMaxBatch];
+        uint16_t *ss[quant::kMaxBatch];
+        int cnt = 0;
+        for (int i = i0; i < count && i < i0 + quant::kMaxBatch; ++i) {
+            if (N[i] == 0) continue;
+            w[cnt] = W[i];
+            k[cnt] = K[i];
+            n[cnt] = N[i];
+            qq[cnt] = q[i];
+            ss[cnt] = scales[i];
+            ++cnt;
+        }
+        if (cnt == 0) continue;
+        rc = w_dtype == W8_F32
+                 ? launch_quantize<float, false, quant::kMaxBatch>(d, cnt, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, k, n, qq, ss, nullptr,
+                                                 INFINITY, st)
+                 : launch_quantize<__half, false, quant::kMaxBatch>(d, cnt, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, k, n, qq, ss, nullptr,
+                                                  INFINITY, st);
+        if (rc != W8_OK) return rc;
+    }
+    return W8_OK;
 }
 
 size_t w8_outlier_capacity(int64_t K, double p) {
