@@ -238,11 +238,12 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *   K % 8 == 0; N >= 1 with N % 8 == 0.  For M <= 64 the number of 8 KB
  *   weight tiles times (multiprocessors + 1) must stay below 2^32 (weights
  *   up to about 230 GB on a B200), else W8_ERR_SHAPE.
- * Stream ordering: for M <= 64 the kernel is launched with programmatic
- *   stream serialization, so its prologue and an L2 prefetch of its first
- *   weight tiles may overlap the previous kernel in the stream; it reads X
- *   and writes Y, the workspace and the counters only after that kernel has
- *   completed, as with an ordinary launch.
+ * Stream ordering: both kernels are launched with programmatic stream
+ *   serialization, so their prologue (and, for M <= 64, an L2 prefetch of
+ *   the first weight tiles) may overlap the previous kernel in the stream;
+ *   they read X, the weights, scales and bias and write Y, the workspace and
+ *   the counters only after that kernel has completed, as with an ordinary
+ *   launch.
  *   workspace  device scratch of at least w8a16_workspace_bytes(M, K, N)
  *              bytes (may be NULL when that is 0).  It must be all zero
  *              before its first use; every call that completes leaves it

@@ -351,6 +351,11 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     }
     tc_fence_before();
     cluster_sync_all();   // barriers initialised in both CTAs, TMEM allocated
+    // The next call may start its prologue as SMs free up.  Every global
+    // access of this call waits for the previous kernel in the stream to
+    // complete: the producers and the epilogue call pdl_wait first (the
+    // converters and the MMA issuer touch only shared and tensor memory).
+    pdl_launch_dependents();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
@@ -360,6 +365,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     if (warp == 0) {
         // ---------------------------------------------------- weight producer
         if (lane == 0) {
+            pdl_wait();
             Ring r;
             int issued = 0;
             bool ok = true;
@@ -391,6 +397,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     } else if (warp == 3) {
         // ---------------------------------------------------- activation producer
         if (lane == 0) {
+            pdl_wait();
             Ring r;
             int issued = 0;
             bool ok = true;
@@ -524,6 +531,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         }
     } else if (warp >= 8) {
         // ---------------------------------------------------- epilogue
+        pdl_wait();
         const int q4 = warp & 3;
         const int half = (warp - 8) >> 2;     // token columns [128 half, 128 half + 128)
         const int r = 32 * q4 + lane;

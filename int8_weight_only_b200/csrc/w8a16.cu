@@ -316,13 +316,17 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
     cfg.blockDim = dim3(prefill2::kThreads, 1, 1);
     cfg.dynamicSmemBytes = prefill2::kSmemBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch: the prologue overlaps the previous
+    // kernel's tail (the kernel waits before every global access)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1;   // the occupancy query takes the cluster shape only
     int resident = 0;
     {
         std::lock_guard<std::mutex> lock(g_mu);
@@ -372,6 +376,7 @@ int launch_prefill2(DeviceInfo *d, const uint16_t *X, const uint8_t *packed, con
         p.sk_iters = 0;
     }
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.numAttrs = 2;
     using namespace prefill2;
     cudaError_t e;
     if (o.count) {
