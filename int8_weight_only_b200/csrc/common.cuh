@@ -241,6 +241,15 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 // 2-D tiled tensor load (box given by the tensor map) at element
 // coordinates (x = innermost, y).  x * element size must be a multiple of
 // 16 bytes; out-of-range elements are filled with zero.
+__device__ __forceinline__ void tma_load_3d(void *dst_smem, const CUtensorMap *map, int32_t x, int32_t y,
+                                            int32_t z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst_smem, const CUtensorMap *map, int32_t x,
                                             int32_t y, uint64_t *bar) {
     asm volatile(

@@ -83,6 +83,10 @@ struct Params {
     const uint16_t *o_vals;      // [N][o_cap] fp16
     int o_cap;
     int64_t K;
+    // 1: tmap_x is the 3-D view X[kb][m][c] = X[m][64 kb + c] (K % 64 == 0),
+    // and a stage's X slices come in one load; 0: the 2-D map, one load per
+    // 64-wide slice
+    int x3;
     int M;
     int64_t N;
     int KB;        // ceil(K / 64)
@@ -221,10 +225,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                 if (!mbar_wait(&empty[stage], phase ^ 1u, SITE_DEC_EMPTY)) break;
                 uint8_t *ws = base + stage * C::kStageBytes;
                 uint8_t *xs = ws + kStageW;
-                mbar_arrive_expect_tx(&full[stage], cnt * (kTileBytes + C::kXBoxBytes));
-                bulk_g2s_hint(ws, p.packed + (size_t)t * kTileBytes, cnt * kTileBytes, &full[stage], policy);
-                for (int j = 0; j < cnt; ++j)
-                    tma_load_2d(xs + j * C::kXBoxBytes, &tmap_x, (int)(kb + j) * 64, 0, &full[stage]);
+                if (p.x3) {
+                    // one box of four 64-wide slices (beyond the last K
+                    // block the fill is zero, and those bytes count too)
+                    mbar_arrive_expect_tx(&full[stage], cnt * kTileBytes + kTilesPerStage * C::kXBoxBytes);
+                    bulk_g2s_hint(ws, p.packed + (size_t)t * kTileBytes, cnt * kTileBytes, &full[stage], policy);
+                    tma_load_3d(xs, &tmap_x, 0, 0, (int)kb, &full[stage]);
+                } else {
+                    mbar_arrive_expect_tx(&full[stage], cnt * (kTileBytes + C::kXBoxBytes));
+                    bulk_g2s_hint(ws, p.packed + (size_t)t * kTileBytes, cnt * kTileBytes, &full[stage], policy);
+                    for (int j = 0; j < cnt; ++j)
+                        tma_load_2d(xs + j * C::kXBoxBytes, &tmap_x, (int)(kb + j) * 64, 0, &full[stage]);
+                }
                 t += cnt;
                 kb += cnt;
                 if (kb == KB) kb = 0;

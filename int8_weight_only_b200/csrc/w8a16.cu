@@ -118,6 +118,22 @@ int make_map_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType dtype, in
     return r == CUDA_SUCCESS ? W8_OK : W8_ERR_CUDA;
 }
 
+// X [M, K] fp16 viewed as [K/64][M][64] (K % 64 == 0): dims {64, M, K/64},
+// strides {2K, 128} bytes, box {64, rows, 4}, 128-byte swizzle.  The image
+// of a box is four consecutive [rows][64] slices, each swizzled as a 2-D
+// box of one slice would be.  Returns false if the driver declines it.
+bool make_map_x3(CUtensorMap *map, const void *X, uint64_t M, uint64_t K, uint32_t rows) {
+    auto fn = encode_fn();
+    if (!fn || K % 64 != 0) return false;
+    cuuint64_t dims[3] = {64, M, K / 64};
+    cuuint64_t strides[2] = {K * 2, 128};
+    cuuint32_t box[3] = {64, rows, 4};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(X), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool overlap(const void *a, size_t an, const void *b, size_t bn) {
@@ -710,9 +726,12 @@ static int linear_common(const uint16_t *X, const uint8_t *packed, const uint16_
     if (M <= decode::kMaxTokens) {
         const int MT = M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8;
         CUtensorMap map;
-        rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
-                         8 * MT, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (rc != W8_OK) return rc;
+        const bool x3 = make_map_x3(&map, X, (uint64_t)M, (uint64_t)K, 8 * MT);
+        if (!x3) {
+            rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64,
+                             8 * MT, CU_TENSOR_MAP_SWIZZLE_128B);
+            if (rc != W8_OK) return rc;
+        }
         decode::Params p;
         p.packed = packed;
         p.scales = scales;
@@ -723,6 +742,7 @@ static int linear_common(const uint16_t *X, const uint8_t *packed, const uint16_
         p.counters = counters;
         p.X = X;
         p.K = K;
+        p.x3 = x3 ? 1 : 0;
         p.o_count = o.count;
         p.o_rows = o.rows;
         p.o_vals = o.vals;
@@ -911,6 +931,7 @@ extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *pack
     p.o_rows = nullptr;
     p.o_vals = nullptr;
     p.o_cap = 0;
+    p.x3 = 0;
     p.bias = bias;
     p.Y = Y;
     p.partials = static_cast<float *>(scratch);
