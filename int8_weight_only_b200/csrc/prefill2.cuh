@@ -353,8 +353,9 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     cluster_sync_all();   // barriers initialised in both CTAs, TMEM allocated
     // The next call may start its prologue as SMs free up.  Every global
     // access of this call waits for the previous kernel in the stream to
-    // complete: the producers and the epilogue call pdl_wait first (the
-    // converters and the MMA issuer touch only shared and tensor memory).
+    // complete: the producers, the epilogue and (for the zero points) the
+    // converters call pdl_wait first (otherwise the converters and the MMA
+    // issuer touch only shared and tensor memory).
     pdl_launch_dependents();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
@@ -472,6 +473,8 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
         Ring wr, ar;
         bool ok = true;
+        // the zero points may have been written by the previous kernel
+        if constexpr (kMode == kZeroPoint) pdl_wait();
         Sched sched(pair0, pstep, p.dp_tiles, p.sk_iters, p.KS);
         Seg sg;
         while (ok && sched.next(sg)) {
