@@ -336,6 +336,19 @@ int w8_device_status(void *stream, uint32_t *out);
  */
 int w8_test_bounded_wait(uint64_t limit_ns, void *stream);
 
+/*
+ * w8_test_set_decode_helper_delay -- test hook for the decode kernel's
+ * split-K bookkeeping on the current device: until set back to 0, each CTA
+ * waits `delay_ns` (0 .. 1e6) before counting the partial sum it publishes
+ * for its first channel block.  That forces the rarely taken paths -- the
+ * previous CTA finishing the shared block through the general last-arriver
+ * path, and a CTA finishing its first block after its own stream -- whose
+ * results must equal the normal ones bit for bit.  Not for production use
+ * (it slows every decode call).  Synchronous; returns W8_OK, W8_ERR_SHAPE
+ * (delay out of range) or W8_ERR_CUDA.
+ */
+int w8_test_set_decode_helper_delay(uint64_t delay_ns);
+
 /* w8_version -- ABI version of this header (major * 100 + minor). */
 int w8_version(void);
 

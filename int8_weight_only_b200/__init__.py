@@ -84,10 +84,12 @@ def load_library():
         lib.w8_error_string.restype = ctypes.c_char_p
         lib.w8_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         lib.w8_test_bounded_wait.argtypes = [ctypes.c_uint64, vp]
+        lib.w8_test_set_decode_helper_delay.argtypes = [ctypes.c_uint64]
         lib.w8_version.argtypes = []
         for f in ("w8_quantize_per_channel", "w8_prepack", "w8_unpack", "w8a16_linear",
                   "w8a16_linear_decode_static",
-                  "w8_device_status", "w8_test_bounded_wait", "w8_version"):
+                  "w8_device_status", "w8_test_bounded_wait", "w8_test_set_decode_helper_delay",
+                  "w8_version"):
             getattr(lib, f).restype = i32
         _lib = lib
         return lib
@@ -455,3 +457,15 @@ def test_bounded_wait(limit_ns: int, device=None):
 
 
 test_bounded_wait.__test__ = False   # not a pytest test
+
+
+def test_set_decode_helper_delay(delay_ns: int, device=None):
+    """Test hook: delay the decode kernel's count of each CTA's first part."""
+    torch = _torch()
+    lib = load_library()
+    dev = device if device is not None else torch.cuda.current_device()
+    with torch.cuda.device(dev):
+        _check(lib.w8_test_set_decode_helper_delay(delay_ns), "w8_test_set_decode_helper_delay")
+
+
+test_set_decode_helper_delay.__test__ = False   # not a pytest test

@@ -27,6 +27,10 @@ enum WaitSite : unsigned {
     SITE_DEC_FULL = 0x21,
     SITE_DEC_FIX = 0x22,
     SITE_DEC_DRAIN = 0x23,
+    SITE_DEC_PUB = 0x24,     // helper: the consumers' first part stored
+    SITE_DEC_START = 0x25,   // consumers: the helper's count of that part
+    SITE_DEC_PRE = 0x26,     // consumers: the helper's look at the next CTA's part
+    SITE_DEC_POLL = 0x27,    // helper: polling for the next CTA's part
     SITE_PF_EMPTY = 0x30,
     SITE_PF_FULL_CVT = 0x31,
     SITE_PF_FULL_MMA = 0x32,
@@ -141,6 +145,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar_addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of a phase (acquire at CTA scope when it reports
+// completion).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }

@@ -30,6 +30,12 @@
 //    first) short-cuts this: when this CTA reaches that block the next CTA
 //    has normally published already, so its part is loaded into registers
 //    during the stream and the block is finished with no fence or atomic.
+//  - The global round trips of a split never stall the stream: a helper
+//    warp counts the part a CTA publishes mid-stream (its first block) and
+//    watches for the next CTA's part of its last block; the consumers only
+//    store their part and read the helper's verdicts, and a CTA that turns
+//    out to be the last contributor of its first block finishes that block
+//    after its stream.
 #pragma once
 
 #include "common.cuh"
@@ -38,7 +44,8 @@ namespace w8 {
 namespace decode {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+// warps 0-7 consumers, warp 8 producer, warp 9 helper
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kTilesPerStage = 4;
 constexpr int kMaxStages = 4;
 constexpr int kTileBytes = 8192;
@@ -67,6 +74,11 @@ struct Cfg {
 constexpr int kMaxPartialFloats = Cfg<8>::kPartialFloats;
 // Partial slot size when at most 16 tokens are allowed.
 constexpr int kPartialFloats16 = Cfg<2>::kPartialFloats;
+
+// Test hook (0 in normal use): the helper waits this long before counting
+// the CTA's first part, so that the next-CTA fallback and the finish of a
+// first block after the stream run deterministically.
+__device__ unsigned long long g_helper_delay_ns = 0;
 
 struct Params {
     const uint8_t *packed;
@@ -158,6 +170,53 @@ __device__ __forceinline__ void store_y(const Params &p, uint32_t b, int warp, i
     }
 }
 
+// Sum of the parts of channel block b held by CTAs jf..jl, added in CTA
+// order whoever finishes the block (so the result does not depend on who
+// does).  The part of CTA `self` comes from `own` when use_own, otherwise
+// it is read back like the others.  Up to kPar parts are loaded together
+// (one L2 round trip).
+template <int MT>
+__device__ __forceinline__ void gather_parts(const Params &p, uint32_t b, uint32_t jf, uint32_t jl, uint32_t self,
+                                             bool use_own, const float (&own)[MT][4], int warp, int lane,
+                                             float (&sum)[MT][4]) {
+    constexpr int kPar = MT <= 2 ? 8 : 2;
+    const uint32_t KB = (uint32_t)p.KB;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sum[mt][e] = 0.0f;
+    for (uint32_t j0 = jf; j0 <= jl; j0 += kPar) {
+        float part[kPar][MT][4];
+#pragma unroll
+        for (int u = 0; u < kPar; ++u) {
+            const uint32_t j = j0 + u;
+            if (j <= jl && !(use_own && j == self)) {
+                const uint32_t sj = (range_start(j, p.T, p.G) / KB == b) ? 2 * j : 2 * j + 1;
+                const float *src = p.partials + (int64_t)sj * Cfg<MT>::kPartialFloats;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        part[u][mt][e] = __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
+            } else {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) part[u][mt][e] = own[mt][e];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kPar; ++u) {
+            if (j0 + u <= jl) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sum[mt][e] += part[u][mt][e];
+            }
+        }
+    }
+}
+
 // Sum the per-k-slice accumulators of each token tile.
 template <int MT, int NS>
 __device__ __forceinline__ void fold(const float (&acc)[MT][NS][4], float (&out)[MT][4]) {
@@ -183,7 +242,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
     __shared__ uint64_t fix_bar;
-    __shared__ int last_flag[2];   // [0]: partner part ready; [1]: last contributor
+    __shared__ int last_flag[2];   // [1]: last contributor (general path)
+    // helper handshakes: pub_bar -- the consumers stored their first part;
+    // start_bar -- the helper counted it (helper_flag[1]: this CTA was the
+    // last contributor); tail_bar -- the consumers reached the last block;
+    // pre_bar -- the helper's verdict on the next CTA's part (helper_flag[0])
+    __shared__ uint64_t pub_bar, start_bar, tail_bar, pre_bar;
+    __shared__ int helper_flag[2];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -191,6 +256,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     const uint32_t KB = (uint32_t)p.KB;
     const uint32_t t_begin = range_start(cta, p.T, p.G);
     const uint32_t t_end = range_start(cta + 1, p.T, p.G);
+    const uint32_t first_b = t_begin / KB;
+    const uint32_t last_b = (t_end - 1) / KB;
+    // The first channel block starts past K block 0 and more work follows:
+    // its part is published mid-stream (the helper counts it).
+    const bool start_pub = (t_begin % KB != 0) && ((first_b + 1) * KB < t_end);
+    // The last channel block, when only its first K blocks are here and the
+    // rest belongs to the next CTA alone (a two-way split with this CTA
+    // holding the part that is streamed last): the next CTA publishes its
+    // part early in its stream, so this CTA can usually pick it up while
+    // streaming its own part and finish the block without any fence or
+    // atomic at the end.
+    const bool tail_pair = (t_end - last_b * KB < KB) && (last_b * KB >= t_begin) &&
+                           owner_of((last_b + 1) * KB - 1, p.T, p.G) == cta + 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -198,6 +276,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             mbar_init(&empty[s], kConsumerWarps);
         }
         mbar_init(&fix_bar, kConsumerWarps * 32);
+        mbar_init(&pub_bar, kConsumerWarps * 32);
+        mbar_init(&start_bar, 1);
+        mbar_init(&tail_bar, 1);
+        mbar_init(&pre_bar, 1);
         fence_barrier_init();
         prefetch_tensormap(&tmap_x);
     }
@@ -253,6 +335,56 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         return;
     }
 
+    if (warp == kConsumerWarps + 1) {
+        // -------------------------------------------------------- helper
+        if (lane == 0 && (start_pub || tail_pair)) {
+            pdl_wait();
+            if (start_pub) {
+                // count the first part once every consumer has stored its
+                // share of it (their arrivals release the stores; the
+                // atomic publishes them at GPU scope)
+                int last = 0;
+                if (mbar_wait_parked(&pub_bar, 0, SITE_DEC_PUB)) {
+                    const unsigned long long delay = g_helper_delay_ns;
+                    if (delay) {
+                        const unsigned long long t1 = globaltimer_ns();
+#pragma unroll 1
+                        while (globaltimer_ns() - t1 < delay) __nanosleep(1000);
+                    }
+                    const uint32_t jf = owner_of(first_b * KB, p.T, p.G);
+                    const uint32_t jl = owner_of((first_b + 1) * KB - 1, p.T, p.G);
+                    const int old = atomic_add_acq_rel_gpu(&p.counters[first_b], 1);
+                    last = ((uint32_t)old == jl - jf);
+                }
+                helper_flag[1] = last;
+                mbar_arrive(&start_bar);
+            }
+            if (tail_pair) {
+                // poll until the next CTA's part is counted, or until the
+                // consumers reach the block (then one last look)
+                int pub = 0;
+                const unsigned long long t0 = globaltimer_ns();
+#pragma unroll 1
+                while (true) {
+                    const bool reached = mbar_test_wait(&tail_bar, 0);
+                    if (ld_acquire_gpu(&p.counters[last_b]) == 1) {
+                        pub = 1;
+                        break;
+                    }
+                    if (reached) break;
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        record_timeout(SITE_DEC_POLL);
+                        break;
+                    }
+                    __nanosleep(256);
+                }
+                helper_flag[0] = pub;
+                mbar_arrive(&pre_bar);
+            }
+        }
+        return;
+    }
+
     // ---------------------------------------------------------- consumers
     pdl_wait();   // before any global access of this grid's consumers
     const int g = lane >> 2, tq = lane & 3;
@@ -287,18 +419,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         return ok;
     };
 
-    // The last channel block of this CTA, when only its first K blocks are
-    // here and the rest belongs to the next CTA alone (a two-way split with
-    // this CTA holding the part that is streamed last): the next CTA
-    // publishes its part early in its stream, so this CTA can usually pick
-    // it up while streaming its own part and finish the block without any
-    // fence or atomic at the end.
-    const uint32_t first_b = t_begin / KB;
-    const uint32_t last_b = (t_end - 1) / KB;
-    const bool tail_pair = (t_end - last_b * KB < KB) && (last_b * KB >= t_begin) &&
-                           owner_of((last_b + 1) * KB - 1, p.T, p.G) == cta + 1;
     float pre[MT][4];
     bool have_pre = false;
+    bool pre_pending = false;   // the helper's verdict on it not read yet
+    // the next CTA's part of the last block, into registers
+    auto load_pre = [&]() {
+        const float *src = p.partials + (int64_t)(2 * (cta + 1)) * C::kPartialFloats;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pre[mt][e] = __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
+    };
 
     int stage = 0;
     uint32_t phase = 0;
@@ -318,18 +449,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                 zc_hi = zp_bias2(n_lo + 8 < p.N ? p.zeros[n_lo + 8] : 0);
             }
             if (tail_pair && b == last_b) {
-                if (threadIdx.x == 0) last_flag[0] = (ld_acquire_gpu(&p.counters[b]) == 1);
-                if (!consumers_sync()) return;
-                have_pre = last_flag[0] != 0;
-                if (have_pre) {
-                    const float *src = p.partials + (int64_t)(2 * (cta + 1)) * C::kPartialFloats;
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            pre[mt][e] = __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
-                }
+                if (threadIdx.x == 0) mbar_arrive(&tail_bar);
+                pre_pending = true;
             }
+        }
+        // the helper's verdict, picked up without waiting; the part itself
+        // then arrives during the rest of the stream
+        if (pre_pending && warp_all(mbar_test_wait(&pre_bar, 0))) {
+            pre_pending = false;
+            have_pre = helper_flag[0] != 0;
+            if (have_pre) load_pre();
         }
         const int cnt = (int)min(min((uint32_t)kTilesPerStage, t_end - t), KB - kb);
         // parked, not spinning: eight warps polling one barrier take issue
@@ -387,6 +516,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         // if it started at K block 0 and reached the end.
         float sum[MT][4];
         fold<MT, NS>(acc, sum);
+        if (!(seg_whole && kb == KB) && pre_pending) {
+            // end of the last block before the verdict was seen (a short
+            // block): wait for it here
+            if (!warp_all(mbar_wait(&pre_bar, 0, SITE_DEC_PRE))) return;
+            pre_pending = false;
+            have_pre = helper_flag[0] != 0;
+            if (have_pre) load_pre();
+        }
         if (seg_whole && kb == KB) {
             store_y<MT>(p, b, warp, lane, sum);
         } else if (have_pre && b == last_b) {
@@ -398,6 +535,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                 for (int e = 0; e < 4; ++e) sum[mt][e] += pre[mt][e];
             store_y<MT>(p, b, warp, lane, sum);
             if (threadIdx.x == 0) p.counters[b] = 0;
+        } else if (start_pub && b == first_b) {
+            // publish the first part and stream on: the helper counts it,
+            // and says after the stream whether this CTA completed the count
+            float *mine = p.partials + (int64_t)(2 * cta) * C::kPartialFloats;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    __stcg(&mine[(warp * 4 * MT + 4 * mt + e) * 32 + lane], sum[mt][e]);
+            mbar_arrive(&pub_bar);
         } else {
             // publish this part; the last contributor to arrive adds all
             // parts in CTA order (independent of arrival order), scales and
@@ -420,48 +567,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             }
             if (!consumers_sync()) return;
             if (last_flag[1]) {
-                // all contributors' parts are loaded together (one L2 round
-                // trip for up to kPar of them), then added in CTA order; this
-                // CTA's own part is still in registers
-                constexpr int kPar = MT <= 2 ? 8 : 2;
+                // this CTA's own part is still in registers
                 float own[MT][4];
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        own[mt][e] = sum[mt][e];
-                        sum[mt][e] = 0.0f;
-                    }
-                for (uint32_t j0 = j_first; j0 <= j_last; j0 += kPar) {
-                    float part[kPar][MT][4];
-#pragma unroll
-                    for (int u = 0; u < kPar; ++u) {
-                        const uint32_t j = j0 + u;
-                        if (j <= j_last && j != cta) {
-                            const uint32_t sj = (range_start(j, p.T, p.G) / KB == b) ? 2 * j : 2 * j + 1;
-                            const float *src = p.partials + (int64_t)sj * C::kPartialFloats;
-#pragma unroll
-                            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    part[u][mt][e] = __ldcg(&src[(warp * 4 * MT + 4 * mt + e) * 32 + lane]);
-                        } else {
-#pragma unroll
-                            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) part[u][mt][e] = own[mt][e];
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < kPar; ++u) {
-                        if (j0 + u <= j_last) {
-#pragma unroll
-                            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) sum[mt][e] += part[u][mt][e];
-                        }
-                    }
-                }
+                    for (int e = 0; e < 4; ++e) own[mt][e] = sum[mt][e];
+                gather_parts<MT>(p, b, j_first, j_last, cta, true, own, warp, lane, sum);
                 store_y<MT>(p, b, warp, lane, sum);
                 if (threadIdx.x == 0) p.counters[b] = 0;
             }
@@ -475,6 +587,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         if (kb == KB) { kb = 0; ++b; }
         seg_whole = true;
         seg_new = true;
+    }
+
+    if (start_pub) {
+        // The helper's count of the first part (normally long done).  If it
+        // completed the count, every other part was already published and
+        // this CTA finishes the block.
+        if (!warp_all(mbar_wait(&start_bar, 0, SITE_DEC_START))) return;
+        if (helper_flag[1]) {
+            const uint32_t jf = owner_of(first_b * KB, p.T, p.G);
+            const uint32_t jl = owner_of((first_b + 1) * KB - 1, p.T, p.G);
+            float none[MT][4] = {};
+            float sum[MT][4];
+            gather_parts<MT>(p, first_b, jf, jl, cta, false, none, warp, lane, sum);
+            store_y<MT>(p, first_b, warp, lane, sum);
+            if (threadIdx.x == 0) p.counters[first_b] = 0;
+        }
     }
 }
 

@@ -828,6 +828,13 @@ int w8_test_bounded_wait(uint64_t limit_ns, void *stream) {
     return launch_status();
 }
 
+int w8_test_set_decode_helper_delay(uint64_t delay_ns) {
+    if (delay_ns > 1000000ull) return W8_ERR_SHAPE;
+    const unsigned long long v = delay_ns;
+    if (cudaMemcpyToSymbol(decode::g_helper_delay_ns, &v, sizeof v) != cudaSuccess) return W8_ERR_CUDA;
+    return W8_OK;
+}
+
 int w8_device_status(void *stream, uint32_t *out) {
     if (!out) return W8_ERR_NULL;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -116,3 +116,10 @@ def test_valid_call_without_gpu_fails_loudly(w8lib):
     assert w8lib.w8a16_linear(A, B, C, None, D, 1, 64, 128, E, 1 << 20, None) == -6
     assert w8lib.w8_quantize_per_channel(A, 0, 64, 128, B, C, None) == -6
     assert w8lib.w8a16_workspace_bytes(1, 64, 128) == 0
+
+
+def test_decode_helper_delay_hook_range(w8lib):
+    # checked on the host before any CUDA call
+    w8lib.w8_test_set_decode_helper_delay.argtypes = [ctypes.c_uint64]
+    assert w8lib.w8_test_set_decode_helper_delay(1_000_001) == -2
+    assert w8lib.w8_test_set_decode_helper_delay(1 << 40) == -2
