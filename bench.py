@@ -31,6 +31,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -62,10 +63,16 @@ def peaks():
 
 
 def kernel_source_hash(names):
+    """Hash of the kernel sources with comments and layout removed: an edit
+    of a comment leaves it (and the committed ncu traffic) valid, any change
+    of code does not."""
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "int8_weight_only_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "int8_weight_only_b200", "csrc", n)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

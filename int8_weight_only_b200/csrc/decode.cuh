@@ -10,8 +10,10 @@
 //    so every SM streams the same number of bytes and no tail wave exists.
 //  - One producer warp per CTA moves each stage (up to 4 tiles = 32 KB, plus
 //    the matching 64-wide slices of X) into a 4-stage shared-memory ring
-//    with one 1-D bulk copy (cp.async.bulk) and 2-D TMA loads; 8 consumer
-//    warps each own 16 of the tile's 128 channels.
+//    with one 1-D bulk copy (cp.async.bulk) for the tiles and one 3-D TMA
+//    load for the four X slices (one 2-D load per slice when K is not a
+//    multiple of 64); 8 consumer warps each own 16 of the tile's 128
+//    channels.
 //  - Consumers widen int8 to fp16 in registers (prmt into the exponent
 //    pattern of 1024, then one fp16x2 subtraction) and accumulate in fp32
 //    with mma.sync m16n8k16 (channels as the MMA rows, tokens as its 8
