@@ -82,6 +82,27 @@ __device__ __forceinline__ int quantize_fast(float w, float inv_s, bool &sure) {
     sure = (fabsf(r) < 126.0f) & (d < 0.5f - 0x1p-13f);
     return __float_as_int(t) - 0x4B400000;
 }
+// The same for a whole row segment, with one decision for all of it: every
+// product is unambiguous exactly when the largest |r| and the largest
+// distance to the nearest integer pass the two tests.  code[e] is the
+// rounding sum's bit pattern, 0x4B400000 + rne(r): its low byte, the only
+// part the packing keeps, is already the code's two's-complement byte
+// (0x4B400000 has a zero low byte).
+template <int kN>
+__device__ __forceinline__ bool quantize_fast_seg(const float (&w)[kN], const float (&inv_s)[kN], int (&code)[kN]) {
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+    float rmax = 0.0f, dmax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < kN; ++e) {
+        const float r = w[e] * inv_s[e];
+        const float t = r + kMagic;
+        dmax = fmaxf(dmax, fabsf(r - (t - kMagic)));
+        rmax = fmaxf(rmax, fabsf(r));
+        code[e] = __float_as_int(t);
+    }
+    return (rmax < 126.0f) & (dmax < 0.5f - 0x1p-13f);
+}
+
 __device__ __forceinline__ int quantize_exact(float w, float s) {
     if (s == 0.0f) return 0;
     const int v = __float2int_rn(__fdiv_rn(w, s));
@@ -425,16 +446,17 @@ quantize_kernel(const __grid_constant__ Params<kCap> p) {
                     const int rloc = rsub + w * B::kSweep;
                     float v[B::kCols];
                     load_seg<T>(box + rloc * B::kRowBytes + 16 * t, v);
-                    int code[B::kCols];
+                    int code[B::kCols];   // codes in the low bytes
                     bool sure = true;
+                    if constexpr (kAsym) {
 #pragma unroll
-                    for (int e = 0; e < B::kCols; ++e) {
-                        bool se;
-                        if constexpr (kAsym)
+                        for (int e = 0; e < B::kCols; ++e) {
+                            bool se;
                             code[e] = quantize_fast_asym(v[e], inv[e], zp[e], se);
-                        else
-                            code[e] = quantize_fast(v[e], inv[e], se);
-                        sure &= se;
+                            sure &= se;
+                        }
+                    } else {
+                        sure = quantize_fast_seg<B::kCols>(v, inv, code);
                     }
                     if (!sure) {   // rare: some product lies near a rounding boundary
 #pragma unroll
