@@ -64,6 +64,15 @@ MUTANTS = {
                                      "vals[n * cap + c] = (uint16_t)(oracle_f32_to_f16(col_buf[k]) & 0xFFFCu);"),
     "asym_linear_scale_by_row": ("acc[col] * (double)oracle_f16_to_f32(scales[col])",
                                  "acc[col] * (double)oracle_f16_to_f32(scales[row])"),
+    # fp16 widening
+    "f16_subnormal_step_halved": ("mag = ldexpf((float)frac, -24);", "mag = ldexpf((float)frac, -25);"),
+    "f16_normal_bias_off_by_one": ("(int)exp - 25);", "(int)exp - 24);"),
+    # more of the variants
+    "outlier_rows_descending": ("        for (int64_t k = 0; k < K; ++k) {\n            /* at most K - r",
+                                "        for (int64_t k = K - 1; k >= 0; --k) {\n            /* at most K - r"),
+    "asym_divide_by_fp32_scale": ("float rr = nearbyintf(col_vals[k] / s);\n            /* |W / S| stays",
+                                  "float rr = nearbyintf(col_vals[k] / (range / 255.0f));\n            /* |W / S| stays"),
+    "asym_zero_point_from_max": ("float t = lo / s;", "float t = hi / s;"),
 }
 
 

@@ -360,6 +360,30 @@ def pin_asym_zero_weight_is_exact_and_sign_ranges(orc):
     assert not q0.any() and not s0.view(np.uint16).any() and not z0.any()
 
 
+def pin_asym_divides_by_the_stored_fp16_scale(orc):
+    # As for the symmetric codes, the weights are divided by the scale that
+    # is stored (fp16), not by the fp32 range / 255 it was rounded from.  A
+    # column over [0, 1] has z = -128 and S = fp16(1/255) != 1/255; one
+    # weight sits where the two scales give different codes.
+    hi = np.float32(1.0)
+    s32 = hi / np.float32(255.0)
+    s16 = np.float32(np.float16(s32))
+    assert s16 != s32
+    # the two scales differ by about 1.5e-5 relatively, so the weight sits
+    # high in the range and within a few thousandths of a half-integer
+    w = by16 = by32 = None
+    for x in (np.float32(200.501), np.float32(200.499), np.float32(240.5015), np.float32(240.4985)):
+        w = x * s16
+        by16, by32 = np.rint(w / s16), np.rint(w / s32)
+        if by16 != by32:
+            break
+    assert by16 != by32                         # the case distinguishes them
+    q, s, z = orc.quantize_asym(np.array([[0.0], [hi], [w]], dtype=np.float32))
+    assert np.float32(s[0]) == s16 and z[0] == -128
+    assert q[1, 0] == 127 and q[0, 0] == -128
+    assert int(q[2, 0]) == int(by16) - 128
+
+
 def pin_asym_reconstruction_error_bound(orc):
     # |w - (q - z) S| <= S / 2, widened by the scale's fp16 rounding, which
     # can stretch the top of the range by up to 255 * 2^-11 of a level
