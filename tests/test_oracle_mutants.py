@@ -73,6 +73,13 @@ MUTANTS = {
     "asym_divide_by_fp32_scale": ("float rr = nearbyintf(col_vals[k] / s);\n            /* |W / S| stays",
                                   "float rr = nearbyintf(col_vals[k] / (range / 255.0f));\n            /* |W / S| stays"),
     "asym_zero_point_from_max": ("float t = lo / s;", "float t = hi / s;"),
+    # clamp and GEMM details
+    "clamp_top_at_128": ("            if (rr > 127.0f) {\n                rr = 127.0f;\n            }\n            if (rr < -127.0f) {",
+                         "            if (rr > 128.0f) {\n                rr = 128.0f;\n            }\n            if (rr < -127.0f) {"),
+    "linear_fp32_accumulation": ("                acc[n] += x * (double)qrow[n];",
+                                 "                acc[n] = (double)(float)(acc[n] + x * (double)qrow[n]);"),
+    "bias_scaled": ("                y += (double)oracle_f16_to_f32(bias[n]);\n            }\n            Y[m * N + n] = y;\n        }\n    }\n}\n\n/* ------",
+                    "                y += (double)oracle_f16_to_f32(bias[n]) * (double)oracle_f16_to_f32(scales[n]);\n            }\n            Y[m * N + n] = y;\n        }\n    }\n}\n\n/* ------"),
 }
 
 
