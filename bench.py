@@ -48,6 +48,8 @@ sys.path.insert(0, ROOT)
 METRIC = "W8A16 GEMM weight GB/s (M=1, 4096×27392) and TFLOP/s (M=2048) on 1 B200"
 K_DIM, N_DIM, M_DECODE, M_PREFILL = 4096, 27392, 1, 2048
 N_COPIES = 6                  # 6 x 112 MB rotating weight copies > 4 x L2
+DECODE_REPS = 60              # timed repetitions behind each median per call
+E2E_GRAPH_STEPS = 48          # end-to-end steps per captured graph
 WORKLOAD = ("chatglm2_h_to_4h_decode: X fp16 [1,4096] . W int8 [4096,27392] "
             "(per-channel int8, fp16 scales), W ~ N(0,0.02) with 0.1% N(0,0.2) outliers")
 FALLBACK_HBM, FALLBACK_TF = 6650.0, 1590.0
@@ -177,8 +179,10 @@ def max_over_ranks(ws, value: float, device) -> float:
     return float(t.item())
 
 
-def timed_replays(graph, n_replays, stream, ws, device, sampler):
-    """Replay `graph` n_replays times between synchronizes; device time in s."""
+def timed_sequence(seq, stream, ws, device, sampler):
+    """Replay each (graph, n) of `seq` n times, in order, between a barrier
+    and a synchronize on both sides; device time in s (CUDA events on the
+    launching stream), max over ranks."""
     import torch
     barrier(ws)
     torch.cuda.synchronize()
@@ -186,14 +190,52 @@ def timed_replays(graph, n_replays, stream, ws, device, sampler):
     t0 = time.time()
     with torch.cuda.stream(stream):
         start.record(stream)
-        for _ in range(n_replays):
-            graph.replay()
+        for graph, n in seq:
+            for _ in range(n):
+                graph.replay()
         end.record(stream)
     torch.cuda.synchronize()
     sampler.mark(t0, time.time())
     elapsed = start.elapsed_time(end) / 1e3
     barrier(ws)
     return max_over_ranks(ws, elapsed, device)
+
+
+def timed_replays(graph, n_replays, stream, ws, device, sampler):
+    """Replay `graph` n_replays times between synchronizes; device time in s."""
+    return timed_sequence([(graph, n_replays)], stream, ws, device, sampler)
+
+
+def replay_times(graph, reps, stream, ws, device, sampler):
+    """Device time (s) of each of `reps` replays of `graph`, CUDA events
+    around every replay on the launching stream; max over ranks per replay."""
+    import torch
+    barrier(ws)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark(t0, time.time())
+    out = [max_over_ranks(ws, a.elapsed_time(b) / 1e3, device) for a, b in evs]
+    barrier(ws)
+    return out
+
+
+# The measured bf16 peaks: a burst (best of 10 GEMMs) and a seconds-long
+# loop under the power cap.  A timed region shorter than SUSTAINED_S is
+# compared with the burst figure.
+SUSTAINED_S = 2.0
+
+
+def tensor_peak(region_s, tf_peak, tf_sustained):
+    if region_s >= SUSTAINED_S and tf_sustained > 0:
+        return tf_sustained, "bf16_tflops_sustained"
+    return tf_peak, "bf16_tflops (burst)"
 
 
 def capture(fn, stream):
@@ -252,19 +294,27 @@ def run_native(args, ws, rank, local):
         for c in copies:
             w8.linear(X1, c, scales, out=Y1, workspace=work)
 
+    # exactly `steps` timed calls: the graph of the 6 copies replayed
+    # steps // 6 times, then a graph of the remaining steps % 6 calls
     g_dec = capture(decode_round, stream)
-    n_rep = -(-steps // N_COPIES)
-    steps_done = n_rep * N_COPIES
+    rem = steps % N_COPIES
+    g_rem = capture(lambda: [w8.linear(X1, c, scales, out=Y1, workspace=work) for c in copies[:rem]],
+                    stream) if rem else None
     for _ in range(max(1, -(-warmup // N_COPIES))):
         with torch.cuda.stream(stream):
             g_dec.replay()
     torch.cuda.synchronize()
-    t_dec = timed_replays(g_dec, n_rep, stream, ws, device, sampler)
+    t_dec = timed_sequence([(g_dec, steps // N_COPIES), (g_rem, 1 if rem else 0)], stream, ws, device, sampler)
+    steps_done = steps
     dec_s = t_dec / steps_done
     weight_bytes = K_DIM * N_DIM
     alg_bytes = weight_bytes + 2 * N_DIM + 2 * M_DECODE * K_DIM + 2 * M_DECODE * N_DIM
     value = ws * weight_bytes * steps_done / t_dec / 1e9
     dec_achieved = alg_bytes / dec_s / 1e9
+    # microseconds per call as the median of DECODE_REPS timed repetitions
+    # (each a replay of the 6-copy graph, CUDA events around it)
+    rep_t = replay_times(g_dec, DECODE_REPS, stream, ws, device, sampler)
+    dec_med_s = statistics.median(rep_t) / N_COPIES
 
     # ---- prefill M = 2048 (two weight copies alternate: 224 MB > L2)
     def prefill_round():
@@ -282,6 +332,8 @@ def run_native(args, ws, rank, local):
     pf_s = t_pf / (2 * n_pf)
     pf_flops = 2.0 * M_PREFILL * K_DIM * N_DIM
     pf_tflops = pf_flops / pf_s / 1e12
+    pf_peak, pf_peak_name = tensor_peak(t_pf, tf_peak, tf_sustained)
+    pf_med_s = statistics.median(replay_times(g_pf, 50, stream, ws, device, sampler)) / 2
 
     # ---- quantize (fp32 W 449 MB > L2) and prepack (one-time weight path)
     q2 = torch.empty_like(q)
@@ -296,31 +348,67 @@ def run_native(args, ws, rank, local):
     n_q = max(5, args.prefill_reps)
     t_q = timed_replays(g_q, n_q, stream, ws, device, sampler) / n_q
     t_pk = timed_replays(g_pk, n_q, stream, ws, device, sampler) / n_q
+    t_q_med = statistics.median(replay_times(g_q, 50, stream, ws, device, sampler))
     q_bytes = K_DIM * N_DIM * (4 + 1) + 2 * N_DIM
     pk_bytes = 2 * K_DIM * N_DIM
     same = bool(torch.equal(q, q2) and torch.equal(scales, s2))
 
-    # ---- e2e: pinned host X -> device, linear, device -> pinned host Y
-    Xh = torch.from_numpy(X1_host).pin_memory()
-    Yh = torch.empty((M_DECODE, N_DIM), dtype=torch.float16).pin_memory()
-    Xd = torch.empty_like(X1)
+    # ---- e2e: per step, the H2D copy of X from pinned host memory, the
+    # public linear call and the D2H copy of Y to pinned host memory.  Two
+    # X and two Y buffers on each side; the copies run on two copy streams
+    # ordered against the compute stream by events, so step i+1's X comes in
+    # and step i's Y goes out while step i or i+1 computes.
+    h2d_stream = torch.cuda.Stream(device)
+    d2h_stream = torch.cuda.Stream(device)
+    Xh = [torch.from_numpy(X1_host).pin_memory() for _ in range(2)]
+    Yh = [torch.empty((M_DECODE, N_DIM), dtype=torch.float16).pin_memory() for _ in range(2)]
+    Xd = [torch.empty_like(X1) for _ in range(2)]
+    Yd = [torch.empty_like(Y1) for _ in range(2)]
 
-    def e2e_round():
-        for c in copies:
-            Xd.copy_(Xh, non_blocking=True)
-            w8.linear(Xd, c, scales, out=Y1, workspace=work)
-            Yh.copy_(Y1, non_blocking=True)
+    def e2e_steps(n):
+        cur = torch.cuda.current_stream(device)
+        h2d_stream.wait_stream(cur)
+        d2h_stream.wait_stream(cur)
+        computed = [None, None]   # compute of the last step that used slot
+        drained = [None, None]    # D2H of the last step that used slot
+        for i in range(n):
+            sl = i % 2
+            if computed[sl] is not None:
+                h2d_stream.wait_event(computed[sl])       # X[sl] no longer read
+            with torch.cuda.stream(h2d_stream):
+                Xd[sl].copy_(Xh[sl], non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(h2d_stream)
+            cur.wait_event(landed)
+            if drained[sl] is not None:
+                cur.wait_event(drained[sl])              # Y[sl] already copied out
+            w8.linear(Xd[sl], copies[i % N_COPIES], scales, out=Yd[sl], workspace=work)
+            computed[sl] = torch.cuda.Event()
+            computed[sl].record(cur)
+            d2h_stream.wait_event(computed[sl])
+            with torch.cuda.stream(d2h_stream):
+                Yh[sl].copy_(Yd[sl], non_blocking=True)
+            drained[sl] = torch.cuda.Event()
+            drained[sl].record(d2h_stream)
+        cur.wait_stream(h2d_stream)
+        cur.wait_stream(d2h_stream)
 
-    g_e2e = capture(e2e_round, stream)
-    for _ in range(3):
+    e2e_full = min(steps, E2E_GRAPH_STEPS)
+    g_e2e = capture(lambda: e2e_steps(e2e_full), stream)
+    e2e_rem = steps % e2e_full
+    g_e2e_rem = capture(lambda: e2e_steps(e2e_rem), stream) if e2e_rem else None
+    for _ in range(2):
         with torch.cuda.stream(stream):
             g_e2e.replay()
     torch.cuda.synchronize()
-    t_e2e = timed_replays(g_e2e, n_rep, stream, ws, device, sampler)
-    e2e_value = ws * weight_bytes * steps_done / t_e2e / 1e9
+    t_e2e = timed_sequence([(g_e2e, steps // e2e_full), (g_e2e_rem, 1 if e2e_rem else 0)],
+                           stream, ws, device, sampler)
+    e2e_value = ws * weight_bytes * steps / t_e2e / 1e9
+    e2e_ok = bool(torch.equal(Yh[0].to(device), Y1) or torch.equal(Yh[1].to(device), Y1))
 
     def graph_time(fn, reps):
-        """Device seconds per call of fn (captured once, replayed)."""
+        """Device seconds per call of fn: captured once, replayed; the median
+        of max(reps, 50) timed replays, CUDA events around each."""
         with torch.cuda.stream(stream):
             fn()
         torch.cuda.synchronize()
@@ -329,7 +417,7 @@ def run_native(args, ws, rank, local):
             with torch.cuda.stream(stream):
                 g.replay()
         torch.cuda.synchronize()
-        t = timed_replays(g, reps, stream, ws, device, sampler) / reps
+        t = statistics.median(replay_times(g, max(reps, 50), stream, ws, device, sampler))
         del g
         return t
 
@@ -339,15 +427,18 @@ def run_native(args, ws, rank, local):
     if not args.no_variants:
         fl_pf = 2.0 * M_PREFILL * K_DIM * N_DIM
         qa, sa, za = w8.quantize_asym(W)
-        pa = [w8.prepack(qa) for _ in range(2)]
+        pa = [w8.prepack(qa) for _ in range(N_COPIES)]
         t_qa = graph_time(lambda: w8.quantize_asym(W, qa, sa, za), 20)
-        t_da = graph_time(lambda: [w8.linear_asym(X1, c, sa, za, out=Y1, workspace=work) for c in pa], 200) / 2
-        t_pa = graph_time(lambda: [w8.linear_asym(Xp, c, sa, za, out=Yp) for c in pa], 20) / 2
+        t_da = graph_time(lambda: [w8.linear_asym(X1, c, sa, za, out=Y1, workspace=work) for c in pa],
+                          DECODE_REPS) / N_COPIES
+        t_pa = graph_time(lambda: [w8.linear_asym(Xp, c, sa, za, out=Yp) for c in pa[:2]], 20) / 2
         variants["asymmetric"] = {
             "quantize_us": round(t_qa * 1e6, 1), "quantize_GBps": round(q_bytes / t_qa / 1e9, 1),
+            "quantize_frac_hbm": round(q_bytes / t_qa / 1e9 / hbm_peak, 4),
             "decode_m1_us": round(t_da * 1e6, 2), "decode_m1_weight_GBps": round(weight_bytes / t_da / 1e9, 1),
             "decode_m1_frac_hbm": round(alg_bytes / t_da / 1e9 / hbm_peak, 4),
-            "prefill_m2048_us": round(t_pa * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_pa / 1e12, 1)}
+            "prefill_m2048_us": round(t_pa * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_pa / 1e12, 1),
+            "prefill_m2048_frac_tensor_burst": round(fl_pf / t_pa / 1e12 / tf_peak, 4)}
         del pa
         qc = torch.empty_like(q)
         sc_ = torch.empty_like(scales)
@@ -359,14 +450,18 @@ def run_native(args, ws, rank, local):
                                        "quantize_GBps": round(q_bytes / t_cp / 1e9, 1),
                                        "passes_over_W": 5}
         qo, so, co, ro, vo = w8.quantize_outliers(W, 0.999)
-        po = [w8.prepack(qo) for _ in range(2)]
+        po = [w8.prepack(qo) for _ in range(N_COPIES)]
         t_qo = graph_time(lambda: w8.quantize_outliers(W, 0.999), 5)
-        t_do = graph_time(lambda: [w8.linear_outliers(X1, c, so, co, ro, vo, out=Y1) for c in po], 200) / 2
-        t_po = graph_time(lambda: [w8.linear_outliers(Xp, c, so, co, ro, vo, out=Yp) for c in po], 20) / 2
+        t_do = graph_time(lambda: [w8.linear_outliers(X1, c, so, co, ro, vo, out=Y1) for c in po],
+                          DECODE_REPS) / N_COPIES
+        t_po = graph_time(lambda: [w8.linear_outliers(Xp, c, so, co, ro, vo, out=Yp) for c in po[:2]], 20) / 2
         variants["outlier_split"] = {
             "p": 0.999, "outliers_per_channel": int(ro.shape[1]), "quantize_us": round(t_qo * 1e6, 1),
             "decode_m1_us": round(t_do * 1e6, 2), "decode_m1_weight_GBps": round(weight_bytes / t_do / 1e9, 1),
-            "prefill_m2048_us": round(t_po * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_po / 1e12, 1)}
+            "decode_m1_frac_hbm": round(alg_bytes / t_do / 1e9 / hbm_peak, 4),
+            "prefill_m2048_us": round(t_po * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_po / 1e12, 1),
+            "prefill_m2048_frac_tensor_burst": round(fl_pf / t_po / 1e12 / tf_peak, 4),
+            "prefill_m2048_vs_plain": round(t_po / pf_med_s, 3)}
         del po, qo, qc
         torch.cuda.empty_cache()
 
@@ -389,7 +484,7 @@ def run_native(args, ws, rank, local):
                 t = graph_time(lambda: [w8.linear(Xs, c, ss, out=Ysw) for c in ps], 20) / ncp
                 tf = 2.0 * Ms * Ks * Ns / t / 1e12
                 row[f"M={Ms}"] = {"us": round(t * 1e6, 1), "TFLOPs": round(tf, 1),
-                                  "frac_tensor_sustained": round(tf / tf_sustained, 4)}
+                                  "frac_tensor_burst": round(tf / tf_peak, 4)}
                 del Xs, Ysw
             prefill_sweep[f"{Ks}x{Ns}"] = row
             del ps, qs
@@ -439,7 +534,8 @@ def run_native(args, ws, rank, local):
                 "quantize_launches": 1,
                 "quantize_one_launch_per_weight_us": round(t_bq1 * 1e6, 1),
                 "linears_us_per_layer": round(t_bl * 1e6 / bw["layers"], 1),
-                "linears_TFLOPs": round(bl_flops / t_bl / 1e12, 1)}
+                "linears_TFLOPs": round(bl_flops / t_bl / 1e12, 1),
+                "linears_frac_tensor_burst": round(bl_flops / t_bl / 1e12 / tf_peak, 4)}
         del pb, Xb, Yb, qb
         torch.cuda.empty_cache()
 
@@ -463,6 +559,7 @@ def run_native(args, ws, rank, local):
             packed_set.append([pd] + [pd.clone() for _ in range(layers - 1)])
             scale_set.append(sd)
         set_bytes = layers * sum(Kd * Nd for Kd, Nd in mats)
+        names = ["qkv", "dense", "h_to_4h", "4h_to_h"]
         for Md in (1, 16):
             Xs = [torch.from_numpy(synthetic.activations(Md, Kd, seed, synthetic.tensor_id(3, Md, i, 1))).to(device)
                   for i, (Kd, Nd) in enumerate(mats)]
@@ -485,7 +582,7 @@ def run_native(args, ws, rank, local):
             torch.cuda.synchronize()
             reps = max(10, args.set_reps)
             t_set = timed_replays(g_set, reps, stream, ws, device, sampler) / reps
-            decode_set[f"M={Md}"] = {
+            entry = {
                 "us_per_layer_set": round(t_set * 1e6, 1),
                 "us_per_layer": round(t_set * 1e6 / layers, 2),
                 "weight_GBps": round(set_bytes / t_set / 1e9, 1),
@@ -493,11 +590,32 @@ def run_native(args, ws, rank, local):
                 "linears": layers * len(mats), "weight_bytes": set_bytes,
             }
             del g_set
+            # per shape: the 28 layers' calls of one matrix in one graph
+            # (28 distinct weights, > L2), median of DECODE_REPS replays
+            for i, (Kd, Nd) in enumerate(mats):
+                def shape_round(i=i):
+                    for layer in range(layers):
+                        w8.linear(Xs[i], packed_set[i][layer], scale_set[i], out=Ys[i], workspace=wsd)
+                g_sh = capture(shape_round, stream)
+                for _ in range(2):
+                    with torch.cuda.stream(stream):
+                        g_sh.replay()
+                torch.cuda.synchronize()
+                t_call = statistics.median(replay_times(g_sh, DECODE_REPS, stream, ws, device, sampler)) / layers
+                alg = Kd * Nd + 2 * Nd + 2 * Md * Kd + 2 * Md * Nd
+                entry[f"{names[i]}_{Kd}x{Nd}"] = {
+                    "us_per_call": round(t_call * 1e6, 2),
+                    "weight_GBps": round(Kd * Nd / t_call / 1e9, 1),
+                    "frac_hbm": round(alg / t_call / 1e9 / hbm_peak, 4),
+                    "algorithmic_bytes": alg}
+                del g_sh
+            decode_set[f"M={Md}"] = entry
         del packed_set
 
     clocks = sampler.stop()
     pf_mhz = sampler.window_mhz(pf_window)
 
+    pf_region_s = t_pf
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -526,34 +644,47 @@ def run_native(args, ws, rank, local):
             "kernel": "w8::decode::decode_kernel<1>",
             "algorithmic_bytes_per_launch": alg_bytes,
             "peak_source": f"{peak_src} hbm_gbs",
+            "achieved_from": f"mean launch time over the {steps_done} timed calls",
+        },
+        "decode": {
+            "us_per_call_median": round(dec_med_s * 1e6, 3),
+            "us_per_call_mean_timed_region": round(dec_s * 1e6, 3),
+            "median_of": f"{DECODE_REPS} timed repetitions of {N_COPIES} calls (one per weight copy)",
+            "weight_GBps_at_median": round(weight_bytes / dec_med_s / 1e9, 1),
+            "frac_hbm_at_median": round(alg_bytes / dec_med_s / 1e9 / hbm_peak, 4),
         },
         "prefill": {
             "metric": "TFLOP/s (M=2048, 4096x27392)", "value": round(pf_tflops, 1), "unit": "TFLOP/s",
             "us_per_call": round(pf_s * 1e6, 2),
+            "us_per_call_median": round(pf_med_s * 1e6, 2),
             "calls_timed": 2 * n_pf,
+            "timed_region_s": round(pf_region_s, 4),
             "sm_mhz_median_in_region": pf_mhz,
-            # the prefill timed region is a long back-to-back loop under the
-            # power cap, the condition of the sustained GEMM measurement
-            "roofline": {"bound": "tensor", "achieved": round(pf_tflops, 1), "peak": tf_sustained,
-                         "unit": "TFLOP/s", "frac": round(pf_tflops / tf_sustained, 4),
-                         "frac_of_burst": round(pf_tflops / tf_peak, 4),
+            "roofline": {"bound": "tensor", "achieved": round(pf_tflops, 1), "peak": pf_peak,
+                         "unit": "TFLOP/s", "frac": round(pf_tflops / pf_peak, 4),
+                         "frac_of_sustained": round(pf_tflops / tf_sustained, 4) if tf_sustained else None,
                          "traffic": measured_traffic("prefill2_kernel", ["prefill2.cuh", "common.cuh"]),
                          "kernel": "w8::prefill2::prefill2_kernel (CTA pairs)",
-                         "peak_source": f"{peak_src} bf16_tflops_sustained (cuBLAS loop under the power cap) "
-                                        f"x fp16/bf16 nominal ratio 1; burst {tf_peak}"},
+                         "peak_source": f"{peak_src} {pf_peak_name} x fp16/bf16 nominal ratio 1 "
+                                        f"(timed region {pf_region_s:.3f} s; the sustained figure "
+                                        f"{tf_sustained} applies to regions of {SUSTAINED_S:.0f} s or more)"},
         },
         "quantize": {
-            "us_per_call": round(t_q * 1e6, 2), "algorithmic_GBps": round(q_bytes / t_q / 1e9, 1),
+            "us_per_call": round(t_q * 1e6, 2), "us_per_call_median": round(t_q_med * 1e6, 2),
+            "algorithmic_GBps": round(q_bytes / t_q / 1e9, 1),
             "frac_hbm": round(q_bytes / t_q / 1e9 / hbm_peak, 4), "bit_identical_rerun": same,
             "traffic": measured_traffic("quantize_kernel", ["quantize.cuh", "common.cuh"]),
         },
         "prepack": {"us_per_call": round(t_pk * 1e6, 2),
                     "algorithmic_GBps": round(pk_bytes / t_pk / 1e9, 1)},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
-                "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()),
-                "how": "public API call per step with pinned-host X->device and Y->host copies, "
-                       "graph-replayed"},
+                "h2d_bytes_per_step": int(Xh[0].numel() * Xh[0].element_size()),
+                "d2h_bytes_per_step": int(Yh[0].numel() * Yh[0].element_size()),
+                "steps": steps, "frac_of_device_value": round(e2e_value / value, 4),
+                "result_read_back_matches": e2e_ok,
+                "how": "per step: pinned-host X -> device copy, the public linear call, device -> pinned-host "
+                       "Y copy; copies on two copy streams, double-buffered, ordered by events; "
+                       f"graphs of {e2e_full} steps"},
         "decode_set": ({"workload": "ChatGLM2-6B decode linears, 28 layers x (QKV 4096x4608, dense 4096x4096, "
                                     "h-to-4h 4096x27392, 4h-to-h 13696x4096), distinct weight buffers, one CUDA graph",
                         **decode_set} if decode_set else None),
@@ -565,8 +696,7 @@ def run_native(args, ws, rank, local):
     }
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
-    for g in (g_dec, g_pf, g_q, g_pk, g_e2e):
-        del g
+    del g_dec, g_rem, g_pf, g_q, g_pk, g_e2e, g_e2e_rem
     return out
 
 
@@ -605,56 +735,198 @@ def run_profile(args):
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_slab(cols: int, seed: int):
-    import synthetic
-    tid = synthetic.tensor_id(2, 0, 0, 0)
-    W = synthetic.weights(K_DIM, N_DIM, seed, tid, outlier_frac=0.001)
-    X = synthetic.activations(M_DECODE, K_DIM, seed, tid + 1)
-    return X, np.ascontiguousarray(W[:, :cols])
+def host_cpu():
+    """(logical CPUs this process may use, CPU model name)."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except Exception:
+        pass
+    return n, model
 
 
-def cpu_baseline(seconds: float):
-    """The CPU oracle as it stands (plain C, one thread) on a column slab of
-    the decode workload, repeated for about `seconds`."""
-    import oracle
-    cols = 4096
-    X, Ws = oracle_slab(cols, 20231002)
-    q, s = oracle.quantize(Ws)
-    t0 = time.perf_counter()
-    reps = 0
+def column_slabs(q, chan, width):
+    """q [K, N] and per-channel arrays cut into contiguous column slabs
+    (done once, before any timing)."""
+    N = q.shape[1]
+    return [(np.ascontiguousarray(q[:, a:min(N, a + width)]),
+             [np.ascontiguousarray(c[a:min(N, a + width)]) for c in chan]) for a in range(0, N, width)]
+
+
+class SlabRunner:
+    """Runs one of the oracle's functions over column slabs on a fixed pool
+    of host threads.  Every output channel of the oracle is computed on its
+    own, so the slabs give the oracle's whole-matrix result; only the wall
+    time depends on the thread count."""
+
+    def __init__(self, threads):
+        from concurrent.futures import ThreadPoolExecutor
+        self.threads = threads
+        self.pool = ThreadPoolExecutor(max_workers=threads) if threads > 1 else None
+
+    def map(self, fn, slabs):
+        if self.pool is None:
+            return [fn(*sl) for sl in slabs]
+        return list(self.pool.map(lambda sl: fn(*sl), slabs))
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.shutdown()
+
+
+def linear_width(K):
+    """Columns per slab: about 1 MB of int8 codes."""
+    return max(64, ((1 << 20) // K) // 64 * 64)
+
+
+def time_repeated(fn, min_s):
+    """Wall seconds per call of fn, repeated until min_s has passed (one
+    untimed call first, unless min_s is 0: then a single timed call)."""
+    if min_s > 0:
+        fn()
+    reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.linear(X, q, s)
+        fn()
         reps += 1
         el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    gbps = K_DIM * cols * reps / el / 1e9
-    return {"value": round(gbps, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{reps} x oracle_linear M=1 on a 4096x{cols} column slab of the "
-                      f"4096x27392 weight ({el:.1f} s, host has {os.cpu_count()} cores)"}
+        if el >= min_s:
+            return el / reps, reps
+
+
+def oracle_quantize_threads(W, runner):
+    import oracle
+    parts = runner.map(lambda w, _: oracle.quantize(w), column_slabs(W, [], 1024))
+    return np.concatenate([p[0] for p in parts], axis=1), np.concatenate([p[1] for p in parts])
+
+
+def oracle_linear_timer(X, q, s, runner):
+    """A callable that runs the oracle's linear X . dequant(q, s) over column
+    slabs prepared once here."""
+    import oracle
+    slabs = column_slabs(q, [s], linear_width(q.shape[0]))
+    return lambda: runner.map(lambda qs, ch: oracle.linear(X, qs, ch[0]), slabs)
+
+
+def cpu_baseline(min_s: float):
+    """The CPU oracle as it stands, timed on this host's cores, on bounded
+    samples of the workloads.  Headline: the decode call (M = 1, 4096 x
+    27392) with the oracle driven over column slabs on every core; beside it
+    one core, and the other workloads: the tiny one, one ChatGLM2 decode
+    layer at M = 16 and the prefill shapes at M = 512."""
+    import oracle
+    import synthetic
+    threads, model = host_cpu()
+    runner, single = SlabRunner(threads), SlabRunner(1)
+    seed = synthetic.SEED
+    tid = synthetic.tensor_id(2, 0, 0, 0)
+    W = synthetic.weights(K_DIM, N_DIM, seed, tid, outlier_frac=0.001)
+    X1 = synthetic.activations(M_DECODE, K_DIM, seed, tid + 1)
+    q, s = oracle_quantize_threads(W, runner)
+    t_all, r_all = time_repeated(oracle_linear_timer(X1, q, s, runner), min_s)
+    slab = 4096
+    t_one, r_one = time_repeated(oracle_linear_timer(X1, q[:, :slab], s[:slab], single), min_s)
+    Wslabs = column_slabs(W, [], 1024)
+    t_q_all, _ = time_repeated(lambda: runner.map(lambda w, _: oracle.quantize(w), Wslabs), min_s / 2)
+    Ws1 = np.ascontiguousarray(W[:, :slab])
+    t_q_one, _ = time_repeated(lambda: oracle.quantize(Ws1), min_s / 2)
+    del Wslabs, Ws1, W
+    out = {"value": round(K_DIM * N_DIM / t_all / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+           "cpu_model": model,
+           "sample": f"{r_all} x oracle linear, M=1, the whole 4096x27392 weight, on column slabs over "
+                     f"{threads} host threads ({r_all * t_all:.1f} s)"}
+    cfg = {
+        "chatglm2_h_to_4h_decode": {
+            "linear_M1_all_cores": {"threads": threads, "ms_per_call": round(t_all * 1e3, 2),
+                                    "weight_GBps": round(K_DIM * N_DIM / t_all / 1e9, 4)},
+            "linear_M1_one_core": {"threads": 1, "sample": f"4096x{slab} column slab",
+                                   "weight_GBps": round(K_DIM * slab / t_one / 1e9, 4)},
+            "quantize_all_cores": {"threads": threads, "ms_per_call": round(t_q_all * 1e3, 1),
+                                   "algorithmic_GBps": round((K_DIM * N_DIM * 5 + 2 * N_DIM) / t_q_all / 1e9, 4)},
+            "quantize_one_core": {"threads": 1, "sample": f"4096x{slab} column slab",
+                                  "algorithmic_GBps": round((K_DIM * slab * 5 + 2 * slab) / t_q_one / 1e9, 4)},
+        }}
+    # tiny workload: quantize + linear, one core
+    Wt = synthetic.weights(256, 512, seed, synthetic.tensor_id(1, 0, 0, 0))
+    Xt = synthetic.activations(4, 256, seed, synthetic.tensor_id(1, 4, 0, 1))
+
+    def tiny():
+        qt, st = oracle.quantize(Wt)
+        oracle.linear(Xt, qt, st)
+
+    t_tiny, _ = time_repeated(tiny, min_s / 4)
+    cfg["tiny"] = {"threads": 1, "us_per_quantize_and_linear": round(t_tiny * 1e6, 1)}
+    # one ChatGLM2 decode layer (4 linears) at M = 16, every core; the h-to-4h
+    # weight above stands in for the layer's (same shape and statistics)
+    mats = synthetic.WORKLOADS["chatglm2_decode_set"]["matrices"]
+    layer, layer_bytes = [], 0
+    for i, (Kd, Nd) in enumerate(mats):
+        if (Kd, Nd) == (K_DIM, N_DIM):
+            qd, sd = q, s
+        else:
+            qd, sd = oracle_quantize_threads(
+                synthetic.weights(Kd, Nd, seed, synthetic.tensor_id(3, 0, i, 0), outlier_frac=0.001), runner)
+        layer.append((qd, sd, oracle_linear_timer(synthetic.activations(16, Kd, seed, synthetic.tensor_id(3, 16, i, 1)),
+                                                  qd, sd, runner)))
+        layer_bytes += Kd * Nd
+    t_layer, _ = time_repeated(lambda: [f() for _, _, f in layer], min_s)
+    cfg["chatglm2_decode_layer_M16"] = {"threads": threads, "ms_per_layer": round(t_layer * 1e3, 1),
+                                        "weight_GBps": round(layer_bytes / t_layer / 1e9, 4)}
+    # prefill at M = 512 on both prefill shapes, every core; the decode-set
+    # weights of the same shapes stand in for the prefill workload's
+    Xp = synthetic.activations(512, K_DIM, seed, synthetic.tensor_id(4, 512, 0, 1))
+    t_p0, _ = time_repeated(oracle_linear_timer(Xp, q, s, runner), 0.0)
+    K4, N4 = mats[3]
+    Xp1 = synthetic.activations(512, K4, seed, synthetic.tensor_id(4, 512, 1, 1))
+    t_p1, _ = time_repeated(oracle_linear_timer(Xp1, layer[3][0], layer[3][1], runner), 0.0)
+    cfg["chatglm2_prefill_M512"] = {
+        "threads": threads,
+        f"{K_DIM}x{N_DIM}": {"s_per_call": round(t_p0, 2), "GFLOPs": round(2 * 512 * K_DIM * N_DIM / t_p0 / 1e9, 2)},
+        f"{K4}x{N4}": {"s_per_call": round(t_p1, 2), "GFLOPs": round(2 * 512 * K4 * N4 / t_p1 / 1e9, 2)},
+        "note": "M=2048 is not timed: it is 4x the M=512 work"}
+    out["configs"] = cfg
+    runner.close()
+    return out
 
 
 def run_reference(args):
-    import oracle
-    cols = args.ref_cols
-    X, Ws = oracle_slab(cols, 20231002)
-    q, s = oracle.quantize(Ws)
+    """The reference arm of this benchmark: the CPU oracle, as it stands, on
+    the headline workload (M = 1, the whole 4096 x 27392 weight per step),
+    driven over column slabs on every host core."""
+    import synthetic
+    threads, model = host_cpu()
+    runner = SlabRunner(threads)
+    tid = synthetic.tensor_id(2, 0, 0, 0)
+    W = synthetic.weights(K_DIM, N_DIM, synthetic.SEED, tid, outlier_frac=0.001)
+    X = synthetic.activations(M_DECODE, K_DIM, synthetic.SEED, tid + 1)
+    q, s = oracle_quantize_threads(W, runner)
+    del W
+    step = oracle_linear_timer(X, q, s, runner)
     for _ in range(args.warmup):
-        oracle.linear(X, q, s)
+        step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.linear(X, q, s)
+        step()
     el = time.perf_counter() - t0
-    value = K_DIM * cols * args.steps / el / 1e9
+    runner.close()
+    value = K_DIM * N_DIM * args.steps / el / 1e9
+    sample = (f"{args.steps} steps, each the oracle's linear over the whole 4096x{N_DIM} weight at M=1, "
+              f"on column slabs over {threads} host threads ({model})")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "M": M_DECODE, "K": K_DIM, "N": N_DIM,
-                   "sample": f"each step: oracle linear over a 4096x{cols} column slab"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{args.steps} steps x 4096x{cols} weight slab, M=1"},
+        "config": {"workload": WORKLOAD, "M": M_DECODE, "K": K_DIM, "N": N_DIM, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "cpu_model": model, "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -667,8 +939,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=60)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--prefill-reps", type=int, default=200)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--ref-cols", type=int, default=2048)
+    ap.add_argument("--cpu-seconds", type=float, default=3.0,
+                    help="minimum seconds per CPU-oracle measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-set", action="store_true",
                     help="skip the 28-layer decode set measurement")

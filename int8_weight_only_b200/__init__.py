@@ -345,17 +345,29 @@ _ws_cache = {}
 
 
 def _workspace(device, nbytes: int):
-    """A zero-filled scratch buffer per device, grown on demand.  The kernels
-    leave it zeroed, so it is reused across calls on one stream."""
+    """The default split-K scratch: one zero-filled buffer per (device,
+    stream), grown on demand.  The kernels leave it zeroed after every
+    completed call, so calls on one stream (which never overlap) reuse it;
+    calls on two streams may overlap on the GPU and so get two buffers."""
     torch = _torch()
     if nbytes == 0:
         return None
-    key = torch.device(device).index
+    dev = torch.device(device)
+    key = (dev.index, torch.cuda.current_stream(dev).cuda_stream)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.zeros((max(nbytes, 1 << 20),), dtype=torch.uint8, device=device)
+        buf = torch.zeros((max(nbytes, 1 << 20),), dtype=torch.uint8, device=dev)
         _ws_cache[key] = buf
     return buf
+
+
+def _reset_workspaces(device_index: int):
+    """Zero every default workspace of a device.  A kernel whose bounded wait
+    gave up may have left split-K counters set; the next call through that
+    workspace would otherwise start from them."""
+    for (dev, _), buf in _ws_cache.items():
+        if dev == device_index:
+            buf.zero_()
 
 
 def linear(X, packed, scales, bias=None, out=None, workspace=None):
@@ -438,13 +450,21 @@ class W8A16Linear:
 
 
 def device_status(device=None) -> int:
-    """Synchronize and read (then clear) the device status word."""
+    """Synchronize and read (then clear) the device status word.  A nonzero
+    value means a bounded device wait gave up; the default workspaces of the
+    device are then zeroed, so later calls without ``workspace=`` start from
+    clean split-K counters (a caller-owned workspace must be zeroed by its
+    owner, as include/w8a16.h states)."""
     torch = _torch()
     lib = load_library()
     dev = device if device is not None else torch.cuda.current_device()
     v = ctypes.c_uint32(0)
     with torch.cuda.device(dev):
         _check(lib.w8_device_status(_stream(dev), ctypes.byref(v)), "w8_device_status")
+        if v.value != 0:
+            # a wait ran out: the default workspaces may hold stale counters
+            _reset_workspaces(torch.device("cuda", torch.cuda.current_device()).index)
+            torch.cuda.synchronize()
     return int(v.value)
 
 

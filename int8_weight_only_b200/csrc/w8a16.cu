@@ -40,10 +40,18 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 
+// A failed runtime call: clear the pending (non-sticky) error so that the
+// caller's next, unrelated CUDA call does not report it, and say so.
+inline int cuda_fail() {
+    cudaGetLastError();
+    return W8_ERR_CUDA;
+}
+
 // Per-device one-time setup: architecture check, SM count, kernel attributes.
 int device_info(DeviceInfo **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W8_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail();
+    if (dev < 0 || dev >= kMaxDevices) return W8_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceInfo &d = g_dev[dev];
     if (!d.ready) {
@@ -51,7 +59,7 @@ int device_info(DeviceInfo **out) {
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return W8_ERR_CUDA;
+            return cuda_fail();
         d.sms = sms;
         d.status = (major == 10 && minor == 0) ? W8_OK : W8_ERR_DEVICE;
         if (d.status == W8_OK) {
@@ -82,7 +90,7 @@ int device_info(DeviceInfo **out) {
             smem((const void *)clip::percentile_quantize_kernel<__half, false>, clip::kSmemBytes);
             smem((const void *)clip::percentile_quantize_kernel<float, true>, clip::kSmemBytes);
             smem((const void *)clip::percentile_quantize_kernel<__half, true>, clip::kSmemBytes);
-            if (e != cudaSuccess) return W8_ERR_CUDA;
+            if (e != cudaSuccess) return cuda_fail();
         }
         d.ready = true;
     }
@@ -831,7 +839,7 @@ int w8_test_bounded_wait(uint64_t limit_ns, void *stream) {
 int w8_test_set_decode_helper_delay(uint64_t delay_ns) {
     if (delay_ns > 1000000ull) return W8_ERR_SHAPE;
     const unsigned long long v = delay_ns;
-    if (cudaMemcpyToSymbol(decode::g_helper_delay_ns, &v, sizeof v) != cudaSuccess) return W8_ERR_CUDA;
+    if (cudaMemcpyToSymbol(decode::g_helper_delay_ns, &v, sizeof v) != cudaSuccess) return cuda_fail();
     return W8_OK;
 }
 
@@ -839,9 +847,9 @@ int w8_device_status(void *stream, uint32_t *out) {
     if (!out) return W8_ERR_NULL;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     unsigned int v = 0, zero = 0;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return W8_ERR_CUDA;
-    if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return W8_ERR_CUDA;
-    if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return W8_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_fail();
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return cuda_fail();
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return cuda_fail();
     *out = v;
     return W8_OK;
 }
@@ -924,10 +932,14 @@ extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *pack
         return W8_ERR_CUDA;
     }
     const int MT = M <= 8 ? 1 : 2;
+    // the same X maps as w8a16_linear: one 3-D load per stage when K % 64 == 0
     CUtensorMap map;
-    rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64, 8 * MT,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-    if (rc != W8_OK) return rc;
+    const bool x3 = make_map_x3(&map, X, (uint64_t)M, (uint64_t)K, 8 * MT);
+    if (!x3) {
+        rc = make_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, 64, 8 * MT,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc != W8_OK) return rc;
+    }
     decode::Params p;
     p.packed = packed;
     p.scales = scales;
@@ -938,7 +950,7 @@ extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *pack
     p.o_rows = nullptr;
     p.o_vals = nullptr;
     p.o_cap = 0;
-    p.x3 = 0;
+    p.x3 = x3 ? 1 : 0;
     p.bias = bias;
     p.Y = Y;
     p.partials = static_cast<float *>(scratch);

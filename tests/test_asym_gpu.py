@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import synthetic
-from tests.gpu_helpers import SEED, assert_close, to_gpu, to_np, w8
+from tests.gpu_helpers import SEED, assert_close, par_linear, par_quantize, to_gpu, to_np, w8
 
 pytestmark = pytest.mark.gpu
 
@@ -110,17 +110,17 @@ def test_linear_asym_exact_integers_bit_exact():
         assert np.array_equal(Yg.view(np.uint16), Yref.astype(np.float16).view(np.uint16)), M
 
 
-def test_linear_asym_chatglm2_h_to_4h_decode_sampled():
+def test_linear_asym_chatglm2_h_to_4h_decode_full():
+    # every code, scale, zero point and output of the headline shape
     K, N = 4096, 27392
     tid = 5400
     W = _weights(K, N, tid)
     X = synthetic.activations(1, K, SEED, tid + 1)
     qg, sg, zg, Yg = _asym_pipeline(W, X)
-    rng = np.random.default_rng(7)
-    cols = np.sort(rng.choice(N, 512, replace=False))
-    qo, so, zo = oracle.quantize_asym(np.ascontiguousarray(W[:, cols]))
-    assert np.array_equal(qg[:, cols], qo) and np.array_equal(zg[cols], zo)
-    assert_close(Yg[:, cols], oracle.linear_asym(X, qo, so, zo), "asym h-to-4h decode")
+    qo, so, zo = par_quantize(W, fn=oracle.quantize_asym)
+    assert np.array_equal(sg.view(np.uint16), so.view(np.uint16))
+    assert np.array_equal(qg, qo) and np.array_equal(zg, zo)
+    assert_close(Yg, par_linear(X, qo, so, zo, fn=oracle.linear_asym), "asym h-to-4h decode")
 
 
 def test_linear_asym_rejects_missing_zeros():

@@ -65,3 +65,28 @@ def test_single_rank_needs_no_process_group():
     assert (ws, rank, local) == (1, 0, 0)
     assert bench.max_over_ranks(1, 0.5, torch.device("cpu")) == 0.5
     bench.barrier(1)
+
+
+def test_tensor_peak_follows_the_region_length():
+    import bench
+    assert bench.tensor_peak(0.14, 1617.4, 1370.6) == (1617.4, "bf16_tflops (burst)")
+    assert bench.tensor_peak(5.0, 1617.4, 1370.6) == (1370.6, "bf16_tflops_sustained")
+    assert bench.tensor_peak(5.0, 1617.4, 0.0)[0] == 1617.4
+
+
+def test_cpu_baseline_slabs_give_the_oracles_whole_result():
+    # the CPU baseline drives the unchanged oracle over column slabs on
+    # several threads; the joined result must be the whole-matrix one
+    import numpy as np
+    import bench
+    import oracle
+    import synthetic
+    W = synthetic.weights(128, 700, 1, 5, outlier_frac=0.01)
+    X = synthetic.activations(3, 128, 1, 6)
+    runner = bench.SlabRunner(4)
+    q, s = bench.oracle_quantize_threads(W, runner)
+    q0, s0 = oracle.quantize(W)
+    assert np.array_equal(q, q0) and np.array_equal(s.view(np.uint16), s0.view(np.uint16))
+    parts = bench.oracle_linear_timer(X, q, s, runner)()
+    runner.close()
+    assert np.array_equal(np.concatenate(parts, axis=1), oracle.linear(X, q0, s0))

@@ -14,9 +14,8 @@ be left at zero (the next undelayed call is identical too)."""
 import numpy as np
 import pytest
 
-import oracle
 import synthetic
-from tests.gpu_helpers import assert_close, to_gpu, to_np, torch_mod, w8
+from tests.gpu_helpers import assert_close, par_linear, par_quantize, to_gpu, to_np, torch_mod, w8
 
 pytestmark = pytest.mark.gpu
 
@@ -79,8 +78,7 @@ def test_delayed_count_gives_identical_bits(M, K, N):
     assert torch.equal(y0, y1), "delayed count changed Y"
     assert torch.equal(y0, y2), "counters not left at zero"
 
-    # and the result is right: sampled columns against the oracle
-    qn, sn = to_np(q), to_np(s)
-    cols = np.unique(np.linspace(0, N - 1, 64).astype(np.int64))
-    y_ref = oracle.linear(X, qn[:, cols], sn[cols], bias[cols])
-    assert_close(to_np(y0)[:, cols], y_ref, f"M={M} K={K} N={N}")
+    # and the result is right: every output against the oracle
+    qo, so = par_quantize(W)
+    assert np.array_equal(to_np(q), qo)
+    assert_close(to_np(y0), par_linear(X, qo, so, bias=bias), f"M={M} K={K} N={N}")

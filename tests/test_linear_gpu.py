@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import synthetic
-from tests.gpu_helpers import SEED, assert_close, gpu_pipeline, to_gpu, to_np, w8
+from tests.gpu_helpers import SEED, assert_close, gpu_pipeline, par_linear, par_quantize, to_gpu, to_np, w8
 
 pytestmark = pytest.mark.gpu
 
@@ -51,17 +51,14 @@ def test_prefill_matches_oracle(M, K, N):
     _check_full(M, K, N, 3000 + K + N + M, bias=(M % 2 == 0))
 
 
-def _sampled_blocks(M, K, N, tid, bias=True, per_block=2, seed=3):
-    """GPU pipeline on the whole problem; the oracle on `per_block` channels
-    of every 128-channel block (all tokens)."""
+def _full(M, K, N, tid, bias=True):
+    """GPU pipeline on the whole problem, every code and output checked
+    against the oracle (run on column slabs in parallel)."""
     W, X, b = _case(M, K, N, tid, bias)
     qg, sg, Yg = gpu_pipeline(W, X, b)
-    rng = np.random.default_rng(seed)
-    cols = np.sort(np.concatenate([blk * 128 + rng.choice(min(128, N - blk * 128), per_block, replace=False)
-                                   for blk in range((N + 127) // 128)]))
-    qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
-    assert np.array_equal(qg[:, cols], qo)
-    assert_close(Yg[:, cols], oracle.linear(X, qo, so, None if b is None else b[cols]), f"M={M} K={K} N={N}")
+    qo, so = par_quantize(W)
+    assert np.array_equal(qg, qo) and np.array_equal(sg.view(np.uint16), so.view(np.uint16))
+    assert_close(Yg, par_linear(X, qo, so, bias=b), f"M={M} K={K} N={N}")
     return Yg
 
 
@@ -74,13 +71,13 @@ def test_prefill_k_split_one_step_shares():
 def test_prefill_k_split_shares_cross_tiles():
     # 16 pair tiles of 32 K steps over 74 pairs: shares of 6 or 7 steps start
     # and end inside tiles (both partial-sum slots in use)
-    _sampled_blocks(300, 8192, 2048, 3910)
+    _full(300, 8192, 2048, 3910)
 
 
 def test_prefill_whole_wave_then_k_split():
     # 150 pair tiles of 32 K steps: one wave of whole tiles, then the K steps
     # of the last 76 tiles split over all pairs
-    _sampled_blocks(3800, 8192, 2560, 3920, per_block=1)
+    _full(3800, 8192, 2560, 3920)
 
 
 def test_prefill_k_split_deterministic():
@@ -98,10 +95,10 @@ def test_prefill_k_split_deterministic():
         assert np.array_equal(Y1.view(np.uint16), Y2.view(np.uint16))
 
 
-def test_prefill_whole_waves_ragged_tail_sampled():
+def test_prefill_whole_waves_ragged_tail():
     # 190 pair tiles of 2 K steps: three waves of whole tiles, the last one
     # partly filled
-    _sampled_blocks(1280, 512, 9728, 3950)
+    _full(1280, 512, 9728, 3950)
 
 
 def test_tiny_workload_both_paths():
@@ -196,61 +193,36 @@ def test_empty_batch():
     Y = m.linear(torch.zeros((0, 64), dtype=torch.float16, device="cuda"), packed, s)
     assert tuple(Y.shape) == (0, 128)
 
-
-# ---------------------------------------------------------------- full-size workloads
-def test_chatglm2_h_to_4h_decode_full():
-    # M = 1, 4096 x 27392, 0.1 % outliers: every output checked
-    tid = synthetic.tensor_id(2, 0, 0, 0)
-    K, N = 4096, 27392
-    W = synthetic.weights(K, N, SEED, tid, outlier_frac=0.001)
-    X = synthetic.activations(1, K, SEED, tid + 1)
-    qg, sg, Yg = gpu_pipeline(W, X)
-    rng = np.random.default_rng(11)
-    cols = np.sort(rng.choice(N, 1024, replace=False))
-    qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
-    assert np.array_equal(qg[:, cols], qo)
-    # the oracle's fp64 product over all channels, with the oracle's codes
-    # for the sampled channels and the same codes elsewhere checked above
-    Yref = oracle.linear(X, qo, so)
-    assert_close(Yg[:, cols], Yref, "h-to-4h decode sample")
-    qall, sall = oracle.quantize(W)
-    assert_close(Yg, oracle.linear(X, qall, sall), "h-to-4h decode all")
+# The full-size workloads (every output of every config) are checked in
+# test_full_size_gpu.py.
 
 
-@pytest.mark.parametrize("M", [1, 2, 4, 8, 16, 32, 64])
-def test_chatglm2_decode_layer_sampled(M):
-    rng = np.random.default_rng(M)
-    for i, (K, N) in enumerate(synthetic.WORKLOADS["chatglm2_decode_set"]["matrices"]):
-        tid = synthetic.tensor_id(3, 0, i, 0)
-        W = synthetic.weights(K, N, SEED, tid, outlier_frac=0.001)
-        X = synthetic.activations(M, K, SEED, synthetic.tensor_id(3, M, i, 1))
-        _, _, Yg = gpu_pipeline(W, X)
-        cols = np.sort(rng.choice(N, 256, replace=False))
-        qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
-        assert_close(Yg[:, cols], oracle.linear(X, qo, so), f"layer matrix {i} M={M}")
-
-
-@pytest.mark.parametrize("M", [512, 1024, 2048])
-def test_chatglm2_prefill_sampled(M):
-    rng = np.random.default_rng(M)
-    for i, (K, N) in enumerate(synthetic.WORKLOADS["chatglm2_prefill"]["matrices"]):
-        tid = synthetic.tensor_id(4, 0, i, 0)
-        W = synthetic.weights(K, N, SEED, tid, outlier_frac=0.001)
-        X = synthetic.activations(M, K, SEED, synthetic.tensor_id(4, M, i, 1))
-        _, _, Yg = gpu_pipeline(W, X)
-        cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 62, replace=False)]))
-        qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
-        assert_close(Yg[:, cols], oracle.linear(X, qo, so), f"prefill matrix {i} M={M}")
-
-
-def test_bert_base_4096_tokens_sampled():
-    rng = np.random.default_rng(5)
-    for i, (K, N) in enumerate(synthetic.WORKLOADS["bert_base_4096_tokens"]["matrices"]):
-        tid = synthetic.tensor_id(5, 0, i, 0)
-        W = synthetic.weights(K, N, SEED, tid)
-        X = synthetic.activations(4096, K, SEED, tid + 1)
-        b = synthetic.bias(N, SEED, tid + 2)
-        _, _, Yg = gpu_pipeline(W, X, b)
-        cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 62, replace=False)]))
-        qo, so = oracle.quantize(np.ascontiguousarray(W[:, cols]))
-        assert_close(Yg[:, cols], oracle.linear(X, qo, so, b[cols]), f"bert matrix {i}")
+def test_default_workspace_per_stream():
+    # calls without workspace= on two streams may overlap on the GPU, so
+    # each stream gets its own default split-K scratch; results on both
+    # streams, launched interleaved, must match the oracle
+    torch = pytest.importorskip("torch")
+    m = w8()
+    shapes = [(1, 4096, 4608), (16, 13696, 4096)]
+    cases = []
+    for i, (M, K, N) in enumerate(shapes):
+        W, X, b = _case(M, K, N, 4100 + i)
+        q, s = m.quantize(to_gpu(W))
+        cases.append((W, X, b, m.prepack(q), s, to_gpu(X), to_gpu(b)))
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [[], []]
+    for rep in range(8):
+        for j, st in enumerate(streams):
+            W, X, b, packed, s, Xg, bg = cases[j]
+            with torch.cuda.stream(st):
+                outs[j].append(m.linear(Xg, packed, s, bg))
+    torch.cuda.synchronize()
+    keys = {k for k in m._ws_cache if k[1] in (streams[0].cuda_stream, streams[1].cuda_stream)}
+    assert len(keys) == 2
+    for j in range(2):
+        W, X, b = cases[j][:3]
+        qo, so = oracle.quantize(W)
+        Yref = oracle.linear(X, qo, so, b)
+        for Y in outs[j]:
+            assert_close(to_np(Y), Yref, f"stream {j}")

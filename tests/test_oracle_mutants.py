@@ -53,6 +53,8 @@ MUTANTS = {
     "percentile_floor_rank": ("double rr = ceil(param * (double)K);", "double rr = floor(param * (double)K);"),
     "percentile_signed_values": ("sort_buf[k] = fabsf(col_vals[k]);", "sort_buf[k] = col_vals[k];"),
     "fixed_clip_ignored": ("if (bound > cf) {", "if (0) {"),
+    "fixed_clip_param_rounded_down": ("float cf = (float)param;",
+                                      "float cf = (float)param; if ((double)cf > param) cf = nextafterf(cf, 0.0f);"),
     "clip_codes_not_clamped": ("rr = clampf_range(rr, -127.0f, 127.0f);", "rr = clampf_range(rr, -128.0f, 127.0f);"),
     # outlier split
     "outlier_at_or_above_bound": ("if (fabsf(col_buf[k]) > cut && c < cap) {",

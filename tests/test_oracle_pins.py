@@ -486,6 +486,38 @@ def pin_fixed_clip_scale_and_codes(orc):
     assert s2[5] == ss[0] and np.array_equal(q2[:, 5], qs[:, 0])
 
 
+def pin_fixed_clip_param_is_an_fp32_value(orc):
+    # The C ABI passes the clip as a double but defines the bound in fp32:
+    # bound = min(max|W|, c) with c = fp32(clip_param).  For fp32 weights a
+    # comparison made in double selects the same bound (no fp32 value lies
+    # strictly between c and fp32(c) on the side that would differ), so what
+    # is pinned is the value the bound takes.  The c used is not an fp32
+    # value; fp32(c) lies just above it, and it is chosen where fp32(c)/127
+    # and the quotient of the fp32 value below fp32(c) round to different
+    # fp16 scales, so a bound that is off by one fp32 step changes the
+    # scale.  A column whose max is exactly fp32(c) lies between c and
+    # fp32(c): it is not clipped.  Clipping a column then equals the plain
+    # quantizer (pinned above) on the same column with its entries clamped
+    # to +-fp32(c).
+    c = 0.0900199469178915
+    c32 = np.float32(c)
+    assert float(c32) != c and float(c32) > c
+    below = np.nextafter(c32, np.float32(0))
+    assert np.float16(c32 / np.float32(127)) != np.float16(below / np.float32(127))
+    W = synthetic.weights(300, 24, SEED, 147, outlier_frac=0.02) * np.float32(4.0)
+    W[7, 3] = c32                       # column 3: max exactly fp32(c)
+    W[:, 3] = np.clip(W[:, 3], -c32, c32)
+    W[:, 9] = np.clip(W[:, 9], -c32, c32) * np.float32(0.5)   # column 9: below c
+    q, s = orc.quantize_clip(W, "fixed", c)
+    q32, s32 = orc.quantize_clip(W, "fixed", float(c32))
+    assert np.array_equal(q, q32) and np.array_equal(s.view(np.uint16), s32.view(np.uint16))
+    qc, sc = orc.quantize(np.clip(W, -c32, c32))
+    assert np.array_equal(q, qc) and np.array_equal(s.view(np.uint16), sc.view(np.uint16))
+    q3, s3 = orc.quantize(np.ascontiguousarray(W[:, 3:4]))
+    assert s[3] == s3[0] and np.array_equal(q[:, 3], q3[:, 0])
+    assert np.sum(np.abs(W).max(axis=0) > c32) >= 20      # most columns are clipped
+
+
 # ---------------------------------------------------------------- outlier split
 # weights above the percentage-clip bound kept apart as fp16, code 0; the
 # rest quantized with that bound.

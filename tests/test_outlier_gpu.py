@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 import synthetic
-from tests.gpu_helpers import SEED, assert_close, to_gpu, to_np, w8
+from tests.gpu_helpers import SEED, assert_close, par_linear, par_quantize, to_gpu, to_np, w8
 
 pytestmark = pytest.mark.gpu
 
@@ -49,18 +49,22 @@ def test_linear_outliers(M, K, N):
     _check(M, K, N, 0.995, 7100 + M + K + N, bias=(M % 2 == 1))
 
 
-def test_linear_outliers_chatglm2_h_to_4h_sampled():
+def test_linear_outliers_chatglm2_h_to_4h_full():
+    # every code, scale, side-list entry and output of the headline shape,
+    # through the weight-streaming (M = 1) and tensor-core (M = 256) paths
     m = w8()
     K, N = 4096, 27392
     W = synthetic.weights(K, N, SEED, 7200, outlier_frac=0.001)
+    q, s, c, r, v = m.quantize_outliers(to_gpu(W), 0.999)
+    o = par_quantize(W, fn=lambda w: oracle.quantize_outliers(w, 0.999))
+    assert np.array_equal(to_np(q), o[0]) and np.array_equal(to_np(s).view(np.uint16), o[1].view(np.uint16))
+    assert np.array_equal(to_np(c), o[2]) and np.array_equal(to_np(r), o[3])
+    assert np.array_equal(to_np(v).view(np.uint16), o[4].view(np.uint16))
+    packed = m.prepack(q)
     for M in (1, 256):
         X = synthetic.activations(M, K, SEED, 7201 + M)
-        q, s, c, r, v = m.quantize_outliers(to_gpu(W), 0.999)
-        Y = to_np(m.linear_outliers(to_gpu(X), m.prepack(q), s, c, r, v))
-        cols = np.sort(np.random.default_rng(M).choice(N, 256, replace=False))
-        o = oracle.quantize_outliers(np.ascontiguousarray(W[:, cols]), 0.999)
-        assert np.array_equal(to_np(c)[cols], o[2]) and np.array_equal(to_np(r)[cols], o[3])
-        assert_close(Y[:, cols], oracle.linear_outliers(X, *o), f"h-to-4h outliers M={M}")
+        Y = to_np(m.linear_outliers(to_gpu(X), packed, s, c, r, v))
+        assert_close(Y, par_linear(X, *o, fn=oracle.linear_outliers), f"h-to-4h outliers M={M}")
 
 
 def test_outlier_capacity_limit():
