@@ -34,7 +34,8 @@ def _weights(K, N, tid, outliers=0.001):
     return W
 
 
-@pytest.mark.parametrize("K,N", [(64, 8), (256, 512), (1000, 264), (4096, 4608), (13696, 256), (300, 27392)])
+@pytest.mark.parametrize("K,N", [(64, 8), (256, 512), (1000, 264), (4096, 4608), (6000, 264), (13696, 256),
+                                 (300, 27392), (20000, 40)])
 @pytest.mark.parametrize("dtype", [np.float32, np.float16])
 def test_quantize_asym_bit_exact(K, N, dtype):
     m = w8()

@@ -1,6 +1,7 @@
 """GPU quantization is bit-exact with the oracle (q and scales), on ragged
 shapes, both weight dtypes, the edge columns the method has, and every
-internal path (resident strip, 16-column strip, two-pass streaming)."""
+cluster split of the K range the kernel takes (1 to 4 CTAs for K <= 8192,
+8 above, rows per CTA ragged at the end)."""
 import numpy as np
 import pytest
 
@@ -10,7 +11,8 @@ from tests.gpu_helpers import SEED, par_quantize, to_gpu, to_np, w8
 
 pytestmark = pytest.mark.gpu
 
-SHAPES = [(256, 512), (1, 8), (7, 24), (63, 136), (65, 264), (200, 40), (1000, 1032), (4096, 512)]
+SHAPES = [(256, 512), (1, 8), (7, 24), (63, 136), (65, 264), (200, 40), (1000, 1032), (4096, 512),
+          (4097, 72), (5000, 136), (8192, 264), (8193, 40), (16384, 64), (16392, 24)]
 
 
 def _gpu_quant(W):
