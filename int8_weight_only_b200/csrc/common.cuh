@@ -31,6 +31,7 @@ enum WaitSite : unsigned {
     SITE_DEC_START = 0x25,   // consumers: the helper's count of that part
     SITE_DEC_PRE = 0x26,     // consumers: the helper's look at the next CTA's part
     SITE_DEC_POLL = 0x27,    // helper: polling for the next CTA's part
+    SITE_DEC_CLUSTER = 0x28, // cluster split: the peers' parts in CTA 0
     SITE_PF_EMPTY = 0x30,
     SITE_PF_FULL_CVT = 0x31,
     SITE_PF_FULL_MMA = 0x32,
@@ -318,6 +319,25 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
     return v;
+}
+// Store four floats (16-byte aligned) into the shared memory of some CTA of
+// the cluster.
+__device__ __forceinline__ void st_dsmem_v4(uint32_t cluster_addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+// Split cluster barrier: every thread of the cluster arrives once (relaxed:
+// the writes to publish are fenced separately, e.g. by
+// fence.mbarrier_init), and a thread that will touch another CTA's shared
+// memory waits for the phase first.  Whole warps (.aligned).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    __syncwarp();
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 // Arrive once on an mbarrier of some CTA of the cluster, releasing this
 // thread's prior writes at cluster scope.

@@ -32,6 +32,12 @@
 //    first) short-cuts this: when this CTA reaches that block the next CTA
 //    has normally published already, so its part is loaded into registers
 //    during the stream and the block is finished with no fence or atomic.
+//  - Few channel blocks (a 4096 x 4096 layer has 32 for 148 SMs): the
+//    cluster form.  A thread-block cluster of C CTAs owns one channel block
+//    and splits its K range evenly; at the end CTAs 1..C-1 store their fp32
+//    parts into CTA 0's shared memory (distributed shared memory) and
+//    arrive on its barrier, and CTA 0 adds the parts in rank order, scales
+//    and stores.  No workspace, no counter, no global round trip.
 //  - The global round trips of a split never stall the stream: a helper
 //    warp counts the part a CTA publishes mid-stream (its first block) and
 //    watches for the next CTA's part of its last block; the consumers only
@@ -53,6 +59,8 @@ constexpr int kMaxStages = 4;
 constexpr int kTileBytes = 8192;
 constexpr int kStageW = kTilesPerStage * kTileBytes;
 constexpr int kMaxTokens = 64;     // MT <= 8 token tiles of 8
+constexpr int kMaxClusterDec = 8;  // CTAs per channel block in the cluster form
+constexpr int kMaxTokensCluster = 16;   // the cluster form takes MT <= 2
 
 // MT = token tiles of 8 (1, 2, 4 or 8: up to 8, 16, 32 or 64 tokens).
 template <int MT>
@@ -68,6 +76,8 @@ struct Cfg {
     // few tokens (otherwise one long mma chain), one when the token tiles
     // already give enough independent chains
     static constexpr int kNS = MT <= 2 ? 4 : 1;
+    // cluster form: the parts of CTAs 1..C-1 in CTA 0, after the ring
+    static constexpr int kSmemBytesCluster = kSmemBytes + (kMaxClusterDec - 1) * kPartialFloats * 4;
 };
 
 // Workspace: [partials: 2 slots per SM, sized for MT = 8][counters: one
@@ -235,10 +245,14 @@ __device__ __forceinline__ void fold(const float (&acc)[MT][NS][4], float (&out)
 
 // kZp: asymmetric codes -- every weight is widened to q - z_n (exact in
 // fp16) instead of q; nothing else changes.
-template <int MT, bool kZp>
+// kCl: the cluster form -- grid = channel blocks x C CTAs, cluster dims
+// (C, 1, 1), C <= kMaxClusterDec, MT <= 2; Cfg::kSmemBytesCluster of
+// dynamic shared memory; the workspace is not used.
+template <int MT, bool kZp, bool kCl = false>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     using C = Cfg<MT>;
+    static_assert(!kCl || MT <= 2, "cluster form: up to 16 tokens");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -256,21 +270,31 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     const int lane = threadIdx.x & 31;
     const uint32_t cta = blockIdx.x;
     const uint32_t KB = (uint32_t)p.KB;
-    const uint32_t t_begin = range_start(cta, p.T, p.G);
-    const uint32_t t_end = range_start(cta + 1, p.T, p.G);
+    // cluster form: rank crank of csz CTAs takes the crank-th of csz even
+    // shares of channel block blockIdx.x / csz
+    uint32_t crank = 0, csz = 1;
+    if constexpr (kCl) {
+        crank = cluster_rank();
+        csz = cluster_size();
+    }
+    const uint32_t t_begin = kCl ? (cta / csz) * KB + crank * KB / csz : range_start(cta, p.T, p.G);
+    const uint32_t t_end = kCl ? (cta / csz) * KB + (crank + 1) * KB / csz : range_start(cta + 1, p.T, p.G);
     const uint32_t first_b = t_begin / KB;
     const uint32_t last_b = (t_end - 1) / KB;
     // The first channel block starts past K block 0 and more work follows:
     // its part is published mid-stream (the helper counts it).
-    const bool start_pub = (t_begin % KB != 0) && ((first_b + 1) * KB < t_end);
+    const bool start_pub = !kCl && (t_begin % KB != 0) && ((first_b + 1) * KB < t_end);
     // The last channel block, when only its first K blocks are here and the
     // rest belongs to the next CTA alone (a two-way split with this CTA
     // holding the part that is streamed last): the next CTA publishes its
     // part early in its stream, so this CTA can usually pick it up while
     // streaming its own part and finish the block without any fence or
     // atomic at the end.
-    const bool tail_pair = (t_end - last_b * KB < KB) && (last_b * KB >= t_begin) &&
+    const bool tail_pair = !kCl && (t_end - last_b * KB < KB) && (last_b * KB >= t_begin) &&
                            owner_of((last_b + 1) * KB - 1, p.T, p.G) == cta + 1;
+    // cluster form: the parts of ranks 1..csz-1, in rank 0 (after the ring)
+    float *red_parts = reinterpret_cast<float *>(base + C::kStages * C::kStageBytes);
+    __shared__ uint64_t red_bar;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -282,10 +306,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         mbar_init(&start_bar, 1);
         mbar_init(&tail_bar, 1);
         mbar_init(&pre_bar, 1);
+        if constexpr (kCl) mbar_init(&red_bar, (csz - 1) * kConsumerWarps * 32);
         fence_barrier_init();
         prefetch_tensormap(&tmap_x);
     }
     __syncthreads();
+    // cluster form: every thread arrives here; a peer waits for the phase
+    // (rank 0's barrier initialised) before its first remote access
+    if constexpr (kCl) cluster_arrive_relaxed();
     // The next call may start as soon as SMs free up; it only touches this
     // call's data after its own pdl_wait.
     pdl_launch_dependents();
@@ -518,6 +546,37 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         // if it started at K block 0 and reached the end.
         float sum[MT][4];
         fold<MT, NS>(acc, sum);
+        if constexpr (kCl) {
+            // the cluster's parts of channel block b, added in rank order in
+            // rank 0 (this is the CTA's only segment)
+            if (csz == 1) {
+                store_y<MT>(p, b, warp, lane, sum);
+            } else if (crank != 0) {
+                cluster_wait();
+                const uint32_t dst =
+                    mapa_shared(smem_u32(red_parts + (crank - 1) * C::kPartialFloats), 0);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+                    st_dsmem_v4(dst + 16u * (uint32_t)((warp * MT + mt) * 32 + lane), sum[mt][0], sum[mt][1],
+                                sum[mt][2], sum[mt][3]);
+                mbar_arrive_cluster(mapa_shared(smem_u32(&red_bar), 0));
+            } else {
+                if (!warp_all(mbar_wait_cluster(&red_bar, 0, SITE_DEC_CLUSTER))) return;
+                for (uint32_t r = 1; r < csz; ++r) {
+                    const float *src = red_parts + (r - 1) * C::kPartialFloats;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const float4 v = *reinterpret_cast<const float4 *>(src + 4 * ((warp * MT + mt) * 32 + lane));
+                        sum[mt][0] += v.x;
+                        sum[mt][1] += v.y;
+                        sum[mt][2] += v.z;
+                        sum[mt][3] += v.w;
+                    }
+                }
+                store_y<MT>(p, b, warp, lane, sum);
+            }
+            break;
+        }
         if (!(seg_whole && kb == KB) && pre_pending) {
             // end of the last block before the verdict was seen (a short
             // block): wait for it here

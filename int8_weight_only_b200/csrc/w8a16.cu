@@ -9,7 +9,9 @@
 #include <cmath>
 #include <cstring>
 #include <climits>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "../../include/w8a16.h"
 #include "common.cuh"
@@ -35,6 +37,9 @@ struct DeviceInfo {
     int qclusters_f16[quant::kMaxCluster + 1] = {};
     int qclusters_asym_f32[quant::kMaxCluster + 1] = {};
     int qclusters_asym_f16[quant::kMaxCluster + 1] = {};
+    // resident clusters of the decode kernel's cluster form, by (kernel,
+    // cluster size) (0 = not yet queried)
+    std::map<std::pair<const void *, int>, int> dclusters;
 };
 
 std::mutex g_mu;
@@ -72,6 +77,10 @@ int device_info(DeviceInfo **out) {
             smem((const void *)decode::decode_kernel<4, false>, decode::Cfg<4>::kSmemBytes);
             smem((const void *)decode::decode_kernel<8, false>, decode::Cfg<8>::kSmemBytes);
             smem((const void *)decode::decode_kernel<1, true>, decode::Cfg<1>::kSmemBytes);
+            smem((const void *)decode::decode_kernel<1, false, true>, decode::Cfg<1>::kSmemBytesCluster);
+            smem((const void *)decode::decode_kernel<2, false, true>, decode::Cfg<2>::kSmemBytesCluster);
+            smem((const void *)decode::decode_kernel<1, true, true>, decode::Cfg<1>::kSmemBytesCluster);
+            smem((const void *)decode::decode_kernel<2, true, true>, decode::Cfg<2>::kSmemBytesCluster);
             smem((const void *)decode::decode_kernel<2, true>, decode::Cfg<2>::kSmemBytes);
             smem((const void *)decode::decode_kernel<4, true>, decode::Cfg<4>::kSmemBytes);
             smem((const void *)decode::decode_kernel<8, true>, decode::Cfg<8>::kSmemBytes);
@@ -241,23 +250,99 @@ int launch_quantize(DeviceInfo *d, int count, const void *const *W, CUtensorMapD
 
 // Programmatic dependent launch: this kernel's prologue and an L2 prefetch
 // of its first weight tiles overlap the previous kernel in the stream.
-template <int MT, bool kZp>
-int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t st) {
+// csz > 0: the cluster form, p.G CTAs in clusters of csz.
+template <int MT, bool kZp, bool kCl>
+int launch_decode(const CUtensorMap &map, const decode::Params &p, cudaStream_t st, int csz) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G, 1, 1);
     cfg.blockDim = dim3(decode::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = decode::Cfg<MT>::kSmemBytes;
+    cfg.dynamicSmemBytes = kCl ? decode::Cfg<MT>::kSmemBytesCluster : decode::Cfg<MT>::kSmemBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = kCl ? csz : 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode::decode_kernel<MT, kZp>, map, p) != cudaSuccess) {
-        cudaGetLastError();
-        return W8_ERR_CUDA;
-    }
+    cfg.numAttrs = kCl ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, decode::decode_kernel<MT, kZp, kCl>, map, p) != cudaSuccess) return cuda_fail();
     return launch_status();
+}
+
+// Clusters of `csz` CTAs of the decode kernel's cluster form that can be
+// resident at once (cached per device).
+template <int MT, bool kZp>
+int decode_resident_clusters(DeviceInfo *d, int csz) {
+    const void *fn = (const void *)decode::decode_kernel<MT, kZp, true>;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int &cached = d->dclusters[{fn, csz}];
+    if (cached == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(csz * d->sms), 1, 1);
+        cfg.blockDim = dim3(decode::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = decode::Cfg<MT>::kSmemBytesCluster;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = csz;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, decode::decode_kernel<MT, kZp, true>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cached = n > 0 ? n : -1;
+    }
+    return cached;
+}
+
+// Cluster size for the cluster form of the decode kernel, 0 for the
+// stream-K form.  The cluster form pays off when the channel blocks are
+// few: one cluster per block, as many CTAs per block as keep every cluster
+// resident at once (one wave), each with at least one K block, and enough
+// CTAs in all to keep HBM busy.
+#ifndef W8_DECODE_CLUSTER_MIN_FILL
+#define W8_DECODE_CLUSTER_MIN_FILL 0.7
+#endif
+template <int MT, bool kZp>
+int decode_cluster_size(DeviceInfo *d, int64_t NB, int64_t KB) {
+    if constexpr (MT > 2) {
+        return 0;
+    } else {
+        for (int c = (int)std::min<int64_t>(decode::kMaxClusterDec, d->sms / std::max<int64_t>(NB, 1)); c >= 2;
+             --c) {
+            if (c > KB) continue;
+            if (decode_resident_clusters<MT, kZp>(d, c) < NB) continue;
+            return (double)(NB * c) >= W8_DECODE_CLUSTER_MIN_FILL * d->sms ? c : 0;
+        }
+        return 0;
+    }
+}
+
+// The decode path of both entry points (w8a16_linear with a workspace,
+// w8a16_linear_decode_static with the static scratch): the same kernel and
+// split for the same shape, so the two give the same bits.  p holds
+// everything but the split (T, G) and the scratch pointers' use.
+template <int MT, bool kZp>
+int launch_decode_any(DeviceInfo *d, const CUtensorMap &map, decode::Params p, int64_t NB, cudaStream_t st) {
+    const int csz = decode_cluster_size<MT, kZp>(d, NB, p.KB);
+    const int64_t T = NB * p.KB;
+    if (csz > 0) {
+        if constexpr (MT <= 2) {
+            p.T = (uint32_t)T;
+            p.G = (uint32_t)(NB * csz);
+            return launch_decode<MT, kZp, true>(map, p, st, csz);
+        }
+    }
+    const int G = (int)std::max<int64_t>(1, std::min<int64_t>(T, d->sms));
+    if ((uint64_t)T * (uint64_t)(G + 1) >= (1ull << 32)) return W8_ERR_SHAPE;
+    p.T = (uint32_t)T;
+    p.G = (uint32_t)G;
+    return launch_decode<MT, kZp, false>(map, p, st, 0);
 }
 
 // Percentile clip (clip.cuh): one persistent CTA per SM, panels of 32
@@ -651,8 +736,6 @@ int w8_unpack(const uint8_t *packed, int64_t K, int64_t N, int8_t *q, void *stre
     return launch_status();
 }
 
-// Decode split: one CTA per SM (never more CTAs than tiles).
-static int decode_grid(int sms, int64_t T) { return (int)std::max<int64_t>(1, std::min<int64_t>(T, sms)); }
 
 // Workspace: [fp32 partial sums][int32 counters].  The partial area is the
 // larger of the two kernels' needs -- decode: 2 slots per SM; prefill: 2
@@ -758,24 +841,19 @@ static int linear_common(const uint16_t *X, const uint8_t *packed, const uint16_
         p.M = (int)M;
         p.N = N;
         p.KB = KB;
-        const int64_t T = NB * KB;
-        const int G = decode_grid(d->sms, T);
-        if ((uint64_t)T * (uint64_t)(G + 1) >= (1ull << 32)) return W8_ERR_SHAPE;
-        p.T = (uint32_t)T;
-        p.G = (uint32_t)G;
         if (asym) {
             switch (MT) {
-                case 1: return launch_decode<1, true>(map, p, st);
-                case 2: return launch_decode<2, true>(map, p, st);
-                case 4: return launch_decode<4, true>(map, p, st);
-                default: return launch_decode<8, true>(map, p, st);
+                case 1: return launch_decode_any<1, true>(d, map, p, NB, st);
+                case 2: return launch_decode_any<2, true>(d, map, p, NB, st);
+                case 4: return launch_decode_any<4, true>(d, map, p, NB, st);
+                default: return launch_decode_any<8, true>(d, map, p, NB, st);
             }
         }
         switch (MT) {
-            case 1: return launch_decode<1, false>(map, p, st);
-            case 2: return launch_decode<2, false>(map, p, st);
-            case 4: return launch_decode<4, false>(map, p, st);
-            default: return launch_decode<8, false>(map, p, st);
+            case 1: return launch_decode_any<1, false>(d, map, p, NB, st);
+            case 2: return launch_decode_any<2, false>(d, map, p, NB, st);
+            case 4: return launch_decode_any<4, false>(d, map, p, NB, st);
+            default: return launch_decode_any<8, false>(d, map, p, NB, st);
         }
     }
 
@@ -958,14 +1036,9 @@ extern "C" int w8a16_linear_decode_static(const uint16_t *X, const uint8_t *pack
     p.M = (int)M;
     p.N = N;
     p.KB = KB;
-    const int64_t T = NB * KB;
-    const int G = decode_grid(d->sms, T);
-    if ((uint64_t)T * (uint64_t)(G + 1) >= (1ull << 32)) return W8_ERR_LIMIT;
-    p.T = (uint32_t)T;
-    p.G = (uint32_t)G;
-    if (MT == 1)
-        decode::decode_kernel<1, false><<<p.G, decode::kThreads, decode::Cfg<1>::kSmemBytes, st>>>(map, p);
-    else
-        decode::decode_kernel<2, false><<<p.G, decode::kThreads, decode::Cfg<2>::kSmemBytes, st>>>(map, p);
-    return launch_status();
+    {
+        const int64_t T = NB * KB;
+        if ((uint64_t)T * (uint64_t)(std::min<int64_t>(T, d->sms) + 1) >= (1ull << 32)) return W8_ERR_LIMIT;
+    }
+    return MT == 1 ? launch_decode_any<1, false>(d, map, p, NB, st) : launch_decode_any<2, false>(d, map, p, NB, st);
 }
