@@ -11,8 +11,12 @@
 //    [r kc, (r+1) kc).  Clusters are persistent (as many as fit at once)
 //    and walk the panels.
 //  - One producer thread per CTA streams each panel's rows twice through
-//    one 4-stage shared-memory ring (two CTAs per SM) with 2-D TMA loads: pass 1 (L2
-//    evict-last) for the column |max|, pass 2 (evict-first) to quantize.
+//    one 3-stage ring of 32 KB slots (two CTAs per SM) with 2-D TMA loads
+//    (one per slot, two for fp16, whose 512-row slot exceeds the 256-row
+//    box limit): pass 1 (L2 evict-last) for the column |max|, pass 2
+//    (evict-first) to quantize.  32 KB slots halve the waits and releases
+//    per byte against 16 KB ones (measured: 171 -> 151 us on fp32
+//    4096 x 27392).
 //    The passes are interleaved one panel apart -- P1(0) P1(1) P2(0) P1(2)
 //    P2(1) ... -- so pass 1 of the next panel streams from HBM while this
 //    panel's maxima are combined, and pass 2 reads L2: the rows held between
@@ -35,13 +39,14 @@ constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr int kPanel = 32;          // columns per panel
-constexpr int kStages = 4;
-constexpr int kBoxBytes = 16384;    // one ring slot
+constexpr int kStages = 3;
+constexpr int kBoxBytes = 32768;    // one ring slot
 constexpr int kSmemBytes = kStages * kBoxBytes + 1024;
 constexpr int kMaxCluster = 8;
 constexpr int kPartBufs = 3;        // partial-maxima buffers (see the exchange)
 
-// Box geometry: 128 fp32 rows or 256 fp16 rows of 32 columns (16 KB).  A
+// Box geometry: 256 fp32 rows or 512 fp16 rows of 32 columns (32 KB),
+// loaded as kLoads TMA boxes of kTmaRows rows (a box has at most 256).  A
 // consumer thread owns one 16-byte segment of a row: 4 fp32 or 8 fp16
 // columns; kThreadsPerRow threads cover a row, kSweep rows per sweep of all
 // consumers, kSweeps sweeps per box.
@@ -51,6 +56,8 @@ struct Box {
     static constexpr int kThreadsPerRow = kPanel / kCols;
     static constexpr int kRowBytes = kPanel * (int)sizeof(T);
     static constexpr int kRows = kBoxBytes / kRowBytes;
+    static constexpr int kTmaRows = kRows < 256 ? kRows : 256;
+    static constexpr int kLoads = kRows / kTmaRows;
     static constexpr int kSweep = kConsumers / kThreadsPerRow;
     static constexpr int kSweeps = kRows / kSweep;
 };
@@ -177,7 +184,7 @@ struct Mat {
 // fold away; kMaxBatch for a batch).
 template <int kCap>
 struct Params {
-    CUtensorMap maps[kCap];   // per weight: W [K, N], box 32 columns x Box<T>::kRows rows
+    CUtensorMap maps[kCap];   // per weight: W [K, N], box 32 columns x Box<T>::kTmaRows rows
     Mat mats[kCap];
     int count;
     int panels;        // all weights' panels, ceil(N / 32) each
@@ -210,7 +217,7 @@ __device__ __forceinline__ PanelRef panel_ref(const Params<kCap> &p, int g, uint
 
 // grid = clusters * C CTAs, cluster dims (C, 1, 1), kThreads threads,
 // kSmemBytes dynamic shared memory.  The tensor map covers W [K, N] with
-// a box of 32 columns x Box<T>::kRows rows, no swizzle.
+// a box of 32 columns x Box<T>::kTmaRows rows, no swizzle.
 //
 // Step j of a CTA (panels P_j = cid + j * clusters):
 //   (a) pass 1 over P_j, partial maxima into part[j % 3];
@@ -285,9 +292,12 @@ quantize_kernel(const __grid_constant__ Params<kCap> p) {
                     for (int i = 0; i < pr.nbox; ++i) {
                         if (!mbar_wait_parked(&empty[s], ph ^ 1u, SITE_Q_EMPTY)) { ok = false; break; }
                         mbar_arrive_expect_tx(&full[s], kBoxBytes);
-                        tma_load_2d_hint(ring + s * kBoxBytes, &p.maps[pr.m], pr.local * kPanel,
-                                         (int32_t)(pr.k_begin + (int64_t)i * B::kRows), &full[s],
-                                         pass == 0 ? keep : drop);
+#pragma unroll
+                        for (int l = 0; l < B::kLoads; ++l)
+                            tma_load_2d_hint(ring + s * kBoxBytes + l * B::kTmaRows * B::kRowBytes, &p.maps[pr.m],
+                                             pr.local * kPanel,
+                                             (int32_t)(pr.k_begin + (int64_t)i * B::kRows + l * B::kTmaRows),
+                                             &full[s], pass == 0 ? keep : drop);
                         ++issued;
                         if (++s == kStages) { s = 0; ph ^= 1u; }
                     }

@@ -193,7 +193,7 @@ int launch_quantize(DeviceInfo *d, int count, const void *const *W, CUtensorMapD
         const int64_t kc = cdiv(cdiv(K[i], C), rows) * rows;
         if (kc > INT32_MAX) return W8_ERR_SHAPE;
         int rc = make_map_2d(&p.maps[i], W[i], dt, (int)sizeof(T), (uint64_t)N[i], (uint64_t)K[i], quant::kPanel,
-                             rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+                             quant::Box<T>::kTmaRows, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (rc != W8_OK) return rc;
         p.mats[i].q = q[i];
         p.mats[i].scales = scales[i];
