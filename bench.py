@@ -702,9 +702,10 @@ def run_native(args, ws, rank, local):
 
 # ------------------------------------------------------------------ profiling driver
 def run_profile(args):
-    """A few plain launches of one kernel on the bench's workload, for ncu
-    captures (no graphs, no timing).  Two packed-weight copies alternate so
-    the weight (2 x 112 MB) is not served from L2."""
+    """A few plain launches of one kernel, for ncu captures (no graphs, no
+    timing): the bench's workload, or the weight shape --profile-shape KxN.
+    Packed-weight copies alternate (at least 2, and enough for more than
+    256 MB), so the weight is not served from L2."""
     import torch
     import synthetic
     import int8_weight_only_b200 as w8
@@ -714,23 +715,25 @@ def run_profile(args):
     w8.load_library()
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
+    K, N = (int(v) for v in args.profile_shape.lower().split("x")) if args.profile_shape else (K_DIM, N_DIM)
     tid = synthetic.tensor_id(2, 0, 0, 0)
-    W = torch.from_numpy(synthetic.weights(K_DIM, N_DIM, synthetic.SEED, tid, outlier_frac=0.001)).to(device)
+    W = torch.from_numpy(synthetic.weights(K, N, synthetic.SEED, tid, outlier_frac=0.001)).to(device)
     q, scales = w8.quantize(W)
-    copies = [w8.prepack(q) for _ in range(2)]
+    ncp = max(2, -(-(256 << 20) // (K * N)))
+    copies = [w8.prepack(q) for _ in range(ncp)]
     M = {"decode": M_DECODE, "decode16": 16, "prefill": M_PREFILL}.get(args.profile, M_DECODE)
-    X = torch.from_numpy(synthetic.activations(M, K_DIM, synthetic.SEED, tid + 1)).to(device)
-    Y = torch.empty((M, N_DIM), dtype=torch.float16, device=device)
+    X = torch.from_numpy(synthetic.activations(M, K, synthetic.SEED, tid + 1)).to(device)
+    Y = torch.empty((M, N), dtype=torch.float16, device=device)
     torch.cuda.synchronize()
     for i in range(args.steps):
         if args.profile in ("decode", "decode16", "prefill"):
-            w8.linear(X, copies[i % 2], scales, out=Y)
+            w8.linear(X, copies[i % ncp], scales, out=Y)
         elif args.profile == "quantize":
             w8.quantize(W, q=q, scales=scales)
         elif args.profile == "prepack":
-            w8.prepack(q, out=copies[i % 2])
+            w8.prepack(q, out=copies[i % ncp])
     torch.cuda.synchronize()
-    print(json.dumps({"profile": args.profile, "launches": args.steps, "M": M, "K": K_DIM, "N": N_DIM}))
+    print(json.dumps({"profile": args.profile, "launches": args.steps, "M": M, "K": K, "N": N}))
     return 0
 
 
@@ -949,6 +952,8 @@ def main():
                     help="skip the variant, prefill-sweep and BERT sections")
     ap.add_argument("--profile", choices=["decode", "decode16", "prefill", "quantize", "prepack"],
                     help="run --steps plain launches of one kernel (for ncu) and exit")
+    ap.add_argument("--profile-shape", default="",
+                    help="weight shape KxN for --profile (default: the bench's 4096x27392)")
     args = ap.parse_args()
     if args.profile:
         return run_profile(args)
