@@ -320,11 +320,15 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
     return v;
 }
-// Store four floats (16-byte aligned) into the shared memory of some CTA of
-// the cluster.
-__device__ __forceinline__ void st_dsmem_v4(uint32_t cluster_addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a), "f"(b), "f"(c),
-                 "f"(d)
+// Asynchronous store of four floats (16-byte aligned) into the shared
+// memory of some CTA of the cluster; its 16 bytes are counted (complete_tx)
+// on that CTA's mbarrier `cluster_bar`, whose phase completes once every
+// expected byte has landed, with no fence on the storing side.
+__device__ __forceinline__ void st_async_dsmem_v4(uint32_t cluster_addr, float a, float b, float c, float d,
+                                                  uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     cluster_addr),
+                 "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
                  : "memory");
 }
 // Split cluster barrier: every thread of the cluster arrives once (relaxed:

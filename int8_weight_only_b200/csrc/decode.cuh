@@ -35,9 +35,10 @@
 //  - Few channel blocks (a 4096 x 4096 layer has 32 for 148 SMs): the
 //    cluster form.  A thread-block cluster of C CTAs owns one channel block
 //    and splits its K range evenly; at the end CTAs 1..C-1 store their fp32
-//    parts into CTA 0's shared memory (distributed shared memory) and
-//    arrive on its barrier, and CTA 0 adds the parts in rank order, scales
-//    and stores.  No workspace, no counter, no global round trip.
+//    parts into CTA 0's shared memory with asynchronous distributed-shared-
+//    memory stores whose bytes complete CTA 0's barrier, and CTA 0 adds the
+//    parts in rank order, scales and stores.  No workspace, no counter, no
+//    global round trip, no fence.
 //  - The global round trips of a split never stall the stream: a helper
 //    warp counts the part a CTA publishes mid-stream (its first block) and
 //    watches for the next CTA's part of its last block; the consumers only
@@ -306,7 +307,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
         mbar_init(&start_bar, 1);
         mbar_init(&tail_bar, 1);
         mbar_init(&pre_bar, 1);
-        if constexpr (kCl) mbar_init(&red_bar, (csz - 1) * kConsumerWarps * 32);
+        if constexpr (kCl) {
+            // one arrival (below) plus the bytes of every peer's part
+            mbar_init(&red_bar, 1);
+            if (crank == 0 && csz > 1)
+                mbar_arrive_expect_tx(&red_bar, (csz - 1) * C::kPartialFloats * (uint32_t)sizeof(float));
+        }
         fence_barrier_init();
         prefetch_tensormap(&tmap_x);
     }
@@ -555,13 +561,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                 cluster_wait();
                 const uint32_t dst =
                     mapa_shared(smem_u32(red_parts + (crank - 1) * C::kPartialFloats), 0);
+                const uint32_t bar0 = mapa_shared(smem_u32(&red_bar), 0);
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
-                    st_dsmem_v4(dst + 16u * (uint32_t)((warp * MT + mt) * 32 + lane), sum[mt][0], sum[mt][1],
-                                sum[mt][2], sum[mt][3]);
-                mbar_arrive_cluster(mapa_shared(smem_u32(&red_bar), 0));
+                    st_async_dsmem_v4(dst + 16u * (uint32_t)((warp * MT + mt) * 32 + lane), sum[mt][0], sum[mt][1],
+                                      sum[mt][2], sum[mt][3], bar0);
             } else {
-                if (!warp_all(mbar_wait_cluster(&red_bar, 0, SITE_DEC_CLUSTER))) return;
+                if (!warp_all(mbar_wait(&red_bar, 0, SITE_DEC_CLUSTER))) return;
                 for (uint32_t r = 1; r < csz; ++r) {
                     const float *src = red_parts + (r - 1) * C::kPartialFloats;
 #pragma unroll
