@@ -18,7 +18,7 @@
 //
 // Roles in each CTA (16 warps):
 //   warp 0      weight producer: bulk copy of this CTA's four 8 KB packed
-//               tiles per 256-wide K step into a local 3-stage ring.
+//               tiles per 256-wide K step into a local 2-stage ring.
 //   warp 3      activation producer: four 2-D TMA loads of this CTA's 128
 //               tokens x 64 X halves per K step into a local 2-stage ring of
 //               64 KB slots; the completion is counted on the FIRST CTA's
@@ -28,7 +28,8 @@
 //   warp 1      (first CTA only) MMA issuer; its commits arrive on the
 //               barriers of both CTAs.
 //   warps 8-15  epilogue: drain this CTA's 128 accumulator lanes, release
-//               the accumulator on the first CTA's barrier, scale, store.
+//               the accumulator on the first CTA's barrier, scale, and store
+//               Y through a shared-memory stage as whole 256-byte rows.
 //   warp 2      tensor-memory allocation for the pair.
 //
 // Schedule.  The pairs are persistent.  Whole tiles go round robin over the
@@ -58,13 +59,20 @@ constexpr int kBTc = kBT / 2;            // tokens held by each CTA
 // hide them; 64- and 128-wide steps left the tensor pipe half and a fifth
 // idle.
 constexpr int kKStep = 4;                // 64-wide K blocks per stage
-constexpr int kWStages = 3;
+// Two weight stages measured as fast as three (and faster on short-K
+// shapes); the 32 KB this frees holds the epilogue's Y stage.
+constexpr int kWStages = 2;
 constexpr int kXStages = 2;
 constexpr int kWTile = 8192;             // packed int8 tile, 128 x 64
 constexpr int kWBytes = kKStep * kWTile;
 constexpr int kXBox = kBTc * 128;        // 128 tokens x 64 fp16
 constexpr int kXBytes = kKStep * kXBox;
-constexpr int kSmemBytes = kXStages * kXBytes + kWStages * kWBytes + 1024;
+// Epilogue stage: per half of the tile's tokens, two buffers of 32 tokens x
+// 128 channels fp16 (8 KB), double-buffered.
+constexpr int kYChunk = 32;
+constexpr int kYStageBytes = kYChunk * kBNc * 2;
+constexpr int kYBytes = 2 * 2 * kYStageBytes;
+constexpr int kSmemBytes = kXStages * kXBytes + kWStages * kWBytes + kYBytes + 1024;
 constexpr int kABuf = 2;                 // A buffers of 32 kKStep columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcol0 = kBT;         // first A buffer column
@@ -312,7 +320,8 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *x_ring = base;                                  // kXStages x 16 KB
-    uint8_t *w_ring = base + kXStages * kXBytes;             // kWStages x 8 KB
+    uint8_t *w_ring = base + kXStages * kXBytes;             // kWStages x 32 KB
+    uint8_t *y_stage = w_ring + kWStages * kWBytes;          // epilogue: 2 halves x 2 x 8 KB
     __shared__ uint64_t w_full[kWStages], w_empty[kWStages];
     __shared__ uint64_t x_full[kXStages], x_empty[kXStages];
     __shared__ uint64_t a_full[kABuf], a_empty[kABuf];
@@ -619,6 +628,9 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                     exn[4 * u + 2] = e4.z;
                     exn[4 * u + 3] = e4.w;
                 }
+                // Y through the shared-memory stage, as in the plain path
+                const int64_t nb0 = blk * kBNc;
+                const int cl = 8 * (lane & 15);
 #pragma unroll
                 for (int cchunk = 0; cchunk < 4; ++cchunk) {
                     float ex[32];
@@ -641,14 +653,18 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                         __syncwarp();
                         if (lane == 0) mbar_arrive_remote(leader(&d_empty));
                     }
-                    if (n_ok) {
+                    uint16_t *stg = reinterpret_cast<uint16_t *>(y_stage + (2 * half + (cchunk & 1)) * kYStageBytes);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int m = m0 + 32 * cchunk + i;
-                            if (m < p.M)
-                                p.Y[(int64_t)m * p.N + n] =
-                                    __half_as_ushort(__float2half_rn(fmaf(__uint_as_float(v[i]), sc, ex[i])));
-                        }
+                    for (int i = 0; i < 32; ++i)
+                        stg[i * kBNc + r] = __half_as_ushort(__float2half_rn(fmaf(__uint_as_float(v[i]), sc, ex[i])));
+                    named_bar_sync(2 + half, 128);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int row = 8 * q4 + 2 * j + (lane >> 4);
+                        const int m = m0 + kYChunk * cchunk + row;
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stg + row * kBNc + cl);
+                        if (m < p.M && nb0 + cl < p.N)
+                            *reinterpret_cast<uint4 *>(p.Y + (int64_t)m * p.N + nb0 + cl) = val;
                     }
                 }
             } else if (sg.slot < 0) {
@@ -669,12 +685,33 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(leader(&d_empty));
-                if (n_ok) {
+                // Y through shared memory: each thread holds one channel of
+                // 128 tokens, so direct stores would be 64 bytes per warp
+                // store, one row apart.  The four warps of a half write a
+                // 32-token chunk as [token][channel] into a stage buffer;
+                // then each warp stores 8 whole token rows (128 channels,
+                // 256 bytes) with 16-byte stores.  Two buffers per half: a
+                // warp refills one only after the barrier of the next
+                // chunk, which every warp passes after its stores from it.
+                const int64_t nb0 = blk * kBNc;               // first channel of the block
+                const int cl = 8 * (lane & 15);               // this lane's 8 channels in a row
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        const int m = m0 + 2 * i;
-                        if (m < p.M) p.Y[(int64_t)m * p.N + n] = (uint16_t)(y2[i] & 0xFFFFu);
-                        if (m + 1 < p.M) p.Y[(int64_t)(m + 1) * p.N + n] = (uint16_t)(y2[i] >> 16);
+                for (int cchunk = 0; cchunk < 4; ++cchunk) {
+                    uint16_t *stg = reinterpret_cast<uint16_t *>(y_stage + (2 * half + (cchunk & 1)) * kYStageBytes);
+#pragma unroll
+                    for (int i = 0; i < kYChunk / 2; ++i) {
+                        const uint32_t w2 = y2[16 * cchunk + i];
+                        stg[(2 * i) * kBNc + r] = (uint16_t)(w2 & 0xFFFFu);
+                        stg[(2 * i + 1) * kBNc + r] = (uint16_t)(w2 >> 16);
+                    }
+                    named_bar_sync(2 + half, 128);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int row = 8 * q4 + 2 * j + (lane >> 4);
+                        const int m = m0 + kYChunk * cchunk + row;
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stg + row * kBNc + cl);
+                        if (m < p.M && nb0 + cl < p.N)
+                            *reinterpret_cast<uint4 *>(p.Y + (int64_t)m * p.N + nb0 + cl) = val;
                     }
                 }
             } else if constexpr (kSplit && kMode != kOutliers) {
