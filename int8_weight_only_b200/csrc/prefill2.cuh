@@ -117,7 +117,7 @@ struct Params {
 };
 
 // Outlier term of one CTA's share of a tile, written while its MMAs run and
-// read back in the drain: [256 epilogue threads][128 tokens] fp32.
+// read back in the drain: [128 tokens][256 epilogue threads] fp32.
 constexpr int kExtraFloats = 32 * kEpiWarps * 128;
 
 // Code forms the converters and the epilogue handle.
@@ -560,8 +560,19 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                 const bool nb_ok = nb < p.N;
                 const float bb = (nb_ok && p.bias) ? __half2float(__ushort_as_half(p.bias[nb])) : 0.0f;
                 const int cnt = nb_ok ? p.o_count[nb] : 0;
-                float4 *dst = reinterpret_cast<float4 *>(p.o_extra + (int64_t)blockIdx.x * kExtraFloats +
-                                                         (threadIdx.x - 256) * 128);
+                // the parked terms are token-major, [token][epilogue thread],
+                // so a warp's access at one token is one 128-byte line
+                float *park = p.o_extra + (int64_t)blockIdx.x * kExtraFloats + (threadIdx.x - 256);
+                // up to four outliers (the common case): their rows and
+                // values are read once for the whole tile
+                int64_t krow[4];
+                float kval[4];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = jj < cnt ? jj : 0;
+                    krow[jj] = (cnt > 0 && cnt <= 4) ? p.o_rows[nb * p.o_cap + j] : 0;
+                    kval[jj] = (jj < cnt && cnt <= 4) ? __half2float(__ushort_as_half(p.o_vals[nb * p.o_cap + j])) : 0.0f;
+                }
                 for (int cchunk = 0; cchunk < 4; ++cchunk) {
                     float ex[32];
 #pragma unroll
@@ -574,8 +585,10 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
 #pragma unroll
                         for (int jj = 0; jj < 4; ++jj) {
                             const int j = j0 + jj < cnt ? j0 + jj : j0;
-                            const int64_t k = p.o_rows[nb * p.o_cap + j];
-                            ov[jj] = j0 + jj < cnt ? __half2float(__ushort_as_half(p.o_vals[nb * p.o_cap + j])) : 0.0f;
+                            const int64_t k = cnt <= 4 ? krow[jj] : p.o_rows[nb * p.o_cap + j];
+                            ov[jj] = cnt <= 4 ? kval[jj]
+                                              : (j0 + jj < cnt ? __half2float(__ushort_as_half(p.o_vals[nb * p.o_cap + j]))
+                                                               : 0.0f);
                             const uint4 *src = reinterpret_cast<const uint4 *>(p.XT + k * p.Mp + mb + 32 * cchunk);
 #pragma unroll
                             for (int u = 0; u < 4; ++u) xv[jj][u] = src[u];
@@ -594,8 +607,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                             }
                     }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        dst[8 * cchunk + u] = make_float4(ex[4 * u], ex[4 * u + 1], ex[4 * u + 2], ex[4 * u + 3]);
+                    for (int i = 0; i < 32; ++i) park[(32 * cchunk + i) * (32 * kEpiWarps)] = ex[i];
                 }
             }
             const bool got = warp_all(mbar_wait(&d_full, it & 1, SITE_P2_DFULL));
@@ -617,17 +629,10 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
             if (kMode == kOutliers && sg.slot < 0) {
                 // the parked terms of chunk c + 1 load while chunk c converts;
                 // each chunk is stored right away (no results held)
-                const float4 *xrow = reinterpret_cast<const float4 *>(
-                    p.o_extra + (int64_t)blockIdx.x * kExtraFloats + (threadIdx.x - 256) * 128);
+                const float *park = p.o_extra + (int64_t)blockIdx.x * kExtraFloats + (threadIdx.x - 256);
                 float exn[32];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float4 e4 = xrow[u];
-                    exn[4 * u] = e4.x;
-                    exn[4 * u + 1] = e4.y;
-                    exn[4 * u + 2] = e4.z;
-                    exn[4 * u + 3] = e4.w;
-                }
+                for (int i = 0; i < 32; ++i) exn[i] = park[i * (32 * kEpiWarps)];
                 // Y through the shared-memory stage, as in the plain path
                 const int64_t nb0 = blk * kBNc;
                 const int cl = 8 * (lane & 15);
@@ -638,13 +643,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
                     for (int i = 0; i < 32; ++i) ex[i] = exn[i];
                     if (cchunk < 3) {
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const float4 e4 = xrow[8 * (cchunk + 1) + u];
-                            exn[4 * u] = e4.x;
-                            exn[4 * u + 1] = e4.y;
-                            exn[4 * u + 2] = e4.z;
-                            exn[4 * u + 3] = e4.w;
-                        }
+                        for (int i = 0; i < 32; ++i) exn[i] = park[(32 * (cchunk + 1) + i) * (32 * kEpiWarps)];
                     }
                     uint32_t v[32];
                     tmem_load_32(lane_addr + 32 * cchunk, v);
