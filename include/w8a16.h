@@ -253,12 +253,15 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *              w8_device_status) the workspace must be zeroed again.
  * Kernel choice (internal): M <= 64 streams the weight once with a
  * split-K kernel on the legacy tensor-core path (HBM-bound up to about 32
- * tokens); larger M runs a tcgen05 tensor-core kernel on pairs of SMs
- * (clusters of two thread blocks) with the widened weight tile held in
- * tensor memory, whole 256 x 256 output tiles per pair where they fill
- * the GPU and a K split over all pairs for the tiles that do not.  Both
- * add a tile's partial sums in a fixed order: results are the same on
- * every call.
+ * tokens): an even split of all tiles over the SMs, or, up to 16 tokens on
+ * weights with few 128-channel blocks, one thread-block cluster per block
+ * whose CTAs add their parts in distributed shared memory (this form does
+ * not touch the workspace); larger M runs a tcgen05 tensor-core kernel on
+ * pairs of SMs (clusters of two thread blocks) with the widened weight
+ * tile held in tensor memory, whole 256 x 256 output tiles per pair where
+ * they fill the GPU and a K split over all pairs for the tiles that do
+ * not.  Every form adds a tile's partial sums in a fixed order: results are
+ * the same on every call.
  * Accuracy: |Y - Y_exact| <= 2^-9 |Y_exact| + 1e-3 rms(Y_exact).
  * Errors: W8_ERR_NULL, W8_ERR_SHAPE, W8_ERR_ALIGN, W8_ERR_WORKSPACE,
  *         W8_ERR_ALIAS, W8_ERR_DEVICE, W8_ERR_CUDA.
@@ -295,6 +298,10 @@ int w8a16_linear_asym(const uint16_t *X, const uint8_t *packed, const uint16_t *
  * this library; every GPU that loads the library holds it until the
  * process exits.  Nothing is allocated or freed by the call.
  *
+ *   The kernel, its split of the weight and the order in which partial
+ *   sums are added are those w8a16_linear takes for the same shape, so the
+ *   two return the same bits; where w8a16_linear's form needs no workspace,
+ *   this one touches no scratch either.
  *   Arguments and results as for w8a16_linear, with these limits:
  *   1 <= M <= 16 (M == 0 is a no-op), N <= W8_STATIC_MAX_N, and the device
  *   has at most W8_STATIC_MAX_SMS multiprocessors.  Beyond them the call
