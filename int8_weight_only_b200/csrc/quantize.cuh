@@ -234,7 +234,13 @@ __device__ __forceinline__ PanelRef panel_ref(const Params<kCap> &p, int g, uint
 // kAsym: the asymmetric form -- pass 1 keeps the column minimum and maximum
 // (both start at 0: the range always holds 0), the exchange combines both,
 // and pass 2 writes clamp(rne(w / s) + z, -128, 127).
-template <typename T, bool kAsym, int kCap>
+// kLag: pass 2 of a panel runs after pass 1 of the next (the order above,
+// which hides the exchange behind the next panel's stream); without it a
+// panel's two passes run back to back, which holds half as many rows in
+// L2 between them.  Clusters of 8 (the tall weights) do better without:
+// 13696 x 4096 fp32 95.7 -> 83.4 us, while 4096 x 27392 (clusters of 4)
+// goes 148.8 -> 152.9 us.
+template <typename T, bool kAsym, int kCap, bool kLag = true>
 __global__ void __launch_bounds__(kThreads, 2)
 quantize_kernel(const __grid_constant__ Params<kCap> p) {
     using B = Box<T>;
@@ -286,7 +292,8 @@ quantize_kernel(const __grid_constant__ Params<kCap> p) {
             for (int j = 0; j <= npan && ok; ++j) {
                 for (int pass = 0; pass < 2 && ok; ++pass) {
                     // pass 0: P1 of panel j; pass 1: P2 of panel j - 1
-                    const int pj = pass == 0 ? j : j - 1;
+                    // (kLag) or of panel j
+                    const int pj = (pass == 0 || !kLag) ? j : j - 1;
                     if (pj < 0 || pj >= npan) continue;
                     const PanelRef pr = panel_ref<B::kRows, kCap>(p, cid + pj * p.clusters, rank);
                     for (int i = 0; i < pr.nbox; ++i) {
@@ -392,14 +399,21 @@ quantize_kernel(const __grid_constant__ Params<kCap> p) {
                     }
                 }
             }
-            if (j == 0) {
-                // (c) for panel 0; nothing to read yet
+            if constexpr (kLag) {
+                if (j == 0) {
+                    // (c) for panel 0; nothing to read yet
+                    if (!csync()) { ok = false; break; }
+                    if (c < (int)csize) mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[0]), (uint32_t)c));
+                    continue;
+                }
+            } else {
+                // (c) publish panel j before combining it
+                if (j >= npan) break;
                 if (!csync()) { ok = false; break; }
-                if (c < (int)csize) mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[0]), (uint32_t)c));
-                continue;
+                if (c < (int)csize) mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[j & 1]), (uint32_t)c));
             }
-            // ---------------- (b) combine the maxima of panel j - 1
-            const int pj = j - 1;
+            // ---------------- (b) combine the maxima of panel j - 1 (kLag) or j
+            const int pj = kLag ? j - 1 : j;
             const PanelRef pr = panel_ref<B::kRows, kCap>(p, cid + pj * p.clusters, rank);
             // this weight's outputs, read from the parameter table once
             const int64_t mN = p.mats[pr.m].N;
@@ -435,7 +449,7 @@ quantize_kernel(const __grid_constant__ Params<kCap> p) {
             // every read of panel j - 1's values is done
             if (!csync()) { ok = false; break; }
             // ---------------- (c) publish panel j
-            if (j < npan && c < (int)csize)
+            if (kLag && j < npan && c < (int)csize)
                 mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[j & 1]), (uint32_t)c));
             // ---------------- (d) pass 2 over panel j - 1 (from L2)
             float sc[B::kCols], inv[B::kCols];

@@ -89,12 +89,16 @@ int device_info(DeviceInfo **out) {
             smem((const void *)prefill2::prefill2_kernel<false, prefill2::kZeroPoint>, prefill2::kSmemBytes);
             smem((const void *)prefill2::prefill2_kernel<true, prefill2::kZeroPoint>, prefill2::kSmemBytes);
             smem((const void *)prefill2::prefill2_kernel<false, prefill2::kOutliers>, prefill2::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<float, false, 1>, quant::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<__half, false, 1>, quant::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<float, true, 1>, quant::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<__half, true, 1>, quant::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<float, false, quant::kMaxBatch>, quant::kSmemBytes);
-            smem((const void *)quant::quantize_kernel<__half, false, quant::kMaxBatch>, quant::kSmemBytes);
+#define W8_Q_SMEM(T, A, CAP)                                                                                  \
+    smem((const void *)quant::quantize_kernel<T, A, CAP, true>, quant::kSmemBytes);                          \
+    smem((const void *)quant::quantize_kernel<T, A, CAP, false>, quant::kSmemBytes);
+            W8_Q_SMEM(float, false, 1)
+            W8_Q_SMEM(__half, false, 1)
+            W8_Q_SMEM(float, true, 1)
+            W8_Q_SMEM(__half, true, 1)
+            W8_Q_SMEM(float, false, quant::kMaxBatch)
+            W8_Q_SMEM(__half, false, quant::kMaxBatch)
+#undef W8_Q_SMEM
             smem((const void *)clip::percentile_quantize_kernel<float, false>, clip::kSmemBytes);
             smem((const void *)clip::percentile_quantize_kernel<__half, false>, clip::kSmemBytes);
             smem((const void *)clip::percentile_quantize_kernel<float, true>, clip::kSmemBytes);
@@ -230,7 +234,8 @@ int launch_quantize(DeviceInfo *d, int count, const void *const *W, CUtensorMapD
         if (cached == 0) {
             cfg.gridDim = dim3((unsigned)(C * d->sms), 1, 1);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, quant::quantize_kernel<T, kAsym, kCap>, &cfg) != cudaSuccess ||
+            if (cudaOccupancyMaxActiveClusters(&n, quant::quantize_kernel<T, kAsym, kCap, true>, &cfg) !=
+                    cudaSuccess ||
                 n < 1) {
                 cudaGetLastError();
                 n = std::max(1, d->sms / C);
@@ -241,7 +246,10 @@ int launch_quantize(DeviceInfo *d, int count, const void *const *W, CUtensorMapD
     }
     p.clusters = (int)std::min<int64_t>(panels, resident);
     cfg.gridDim = dim3((unsigned)(p.clusters * C), 1, 1);
-    if (cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T, kAsym, kCap>, p) != cudaSuccess) {
+    // clusters of 8 (tall weights): each panel's passes back to back
+    const cudaError_t le = C == quant::kMaxCluster ? cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T, kAsym, kCap, false>, p)
+                                                   : cudaLaunchKernelEx(&cfg, quant::quantize_kernel<T, kAsym, kCap, true>, p);
+    if (le != cudaSuccess) {
         cudaGetLastError();
         return W8_ERR_CUDA;
     }
