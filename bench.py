@@ -329,25 +329,6 @@ def run_native(args, ws, rank, local):
     rep_t = replay_times(g_dec, DECODE_REPS, stream, ws, device, sampler)
     dec_med_s = statistics.median(rep_t) / N_COPIES
 
-    # ---- prefill M = 2048 (two weight copies alternate: 224 MB > L2)
-    def prefill_round():
-        for c in copies[:2]:
-            w8.linear(Xp, c, scales, out=Yp)
-
-    g_pf = capture(prefill_round, stream)
-    for _ in range(3):
-        with torch.cuda.stream(stream):
-            g_pf.replay()
-    torch.cuda.synchronize()
-    n_pf = max(5, args.prefill_reps)
-    t_pf = timed_replays(g_pf, n_pf, stream, ws, device, sampler)
-    pf_window = sampler.windows[-1]
-    pf_s = t_pf / (2 * n_pf)
-    pf_flops = 2.0 * M_PREFILL * K_DIM * N_DIM
-    pf_tflops = pf_flops / pf_s / 1e12
-    pf_peak, pf_peak_name = tensor_peak(t_pf, tf_peak, tf_sustained)
-    pf_med_s = statistics.median(replay_times(g_pf, 50, stream, ws, device, sampler)) / 2
-
     # ---- quantize (fp32 W 449 MB > L2) and prepack (one-time weight path)
     q2 = torch.empty_like(q)
     s2 = torch.empty_like(scales)
@@ -438,24 +419,22 @@ def run_native(args, ws, rank, local):
         return t
 
     # ---- the method's variants on the headline weight (4096 x 27392, 0.1 %
-    # outliers): asymmetric codes, clipped scales, the outlier split
+    # outliers): asymmetric codes, clipped scales, the outlier split.  Their
+    # memory-bound calls (quantizers, decode) are timed here, before the
+    # prefill loop; their prefill calls after it.
     variants = {}
     if not args.no_variants:
-        fl_pf = 2.0 * M_PREFILL * K_DIM * N_DIM
         qa, sa, za = w8.quantize_asym(W)
         pa = [w8.prepack(qa) for _ in range(N_COPIES)]
         t_qa = graph_time(lambda: w8.quantize_asym(W, qa, sa, za), 20)
         t_da = graph_time(lambda: [w8.linear_asym(X1, c, sa, za, out=Y1, workspace=work) for c in pa],
                           DECODE_REPS) / N_COPIES
-        t_pa = graph_time(lambda: [w8.linear_asym(Xp, c, sa, za, out=Yp) for c in pa[:2]], 20) / 2
         variants["asymmetric"] = {
             "quantize_us": round(t_qa * 1e6, 1), "quantize_GBps": round(q_bytes / t_qa / 1e9, 1),
             "quantize_frac_hbm": round(q_bytes / t_qa / 1e9 / hbm_peak, 4),
             "decode_m1_us": round(t_da * 1e6, 2), "decode_m1_weight_GBps": round(weight_bytes / t_da / 1e9, 1),
-            "decode_m1_frac_hbm": round(alg_bytes / t_da / 1e9 / hbm_peak, 4),
-            "prefill_m2048_us": round(t_pa * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_pa / 1e12, 1),
-            "prefill_m2048_frac_tensor_burst": round(fl_pf / t_pa / 1e12 / tf_peak, 4)}
-        del pa
+            "decode_m1_frac_hbm": round(alg_bytes / t_da / 1e9 / hbm_peak, 4)}
+        del pa[2:]
         qc = torch.empty_like(q)
         sc_ = torch.empty_like(scales)
         t_cf = graph_time(lambda: w8.quantize_clip(W, "fixed", 0.05, qc, sc_), 20)
@@ -464,21 +443,58 @@ def run_native(args, ws, rank, local):
                                   "quantize_GBps": round(q_bytes / t_cf / 1e9, 1)}
         variants["clip_percentile"] = {"p": 0.999, "quantize_us": round(t_cp * 1e6, 1),
                                        "quantize_GBps": round(q_bytes / t_cp / 1e9, 1),
-                                       "passes_over_W": 5}
+                                       "quantize_frac_hbm": round(q_bytes / t_cp / 1e9 / hbm_peak, 4)}
         qo, so, co, ro, vo = w8.quantize_outliers(W, 0.999)
         po = [w8.prepack(qo) for _ in range(N_COPIES)]
         t_qo = graph_time(lambda: w8.quantize_outliers(W, 0.999), 5)
         t_do = graph_time(lambda: [w8.linear_outliers(X1, c, so, co, ro, vo, out=Y1) for c in po],
                           DECODE_REPS) / N_COPIES
-        t_po = graph_time(lambda: [w8.linear_outliers(Xp, c, so, co, ro, vo, out=Yp) for c in po[:2]], 20) / 2
         variants["outlier_split"] = {
             "p": 0.999, "outliers_per_channel": int(ro.shape[1]), "quantize_us": round(t_qo * 1e6, 1),
             "decode_m1_us": round(t_do * 1e6, 2), "decode_m1_weight_GBps": round(weight_bytes / t_do / 1e9, 1),
-            "decode_m1_frac_hbm": round(alg_bytes / t_do / 1e9 / hbm_peak, 4),
+            "decode_m1_frac_hbm": round(alg_bytes / t_do / 1e9 / hbm_peak, 4)}
+        del po[2:], qo, qc
+        torch.cuda.empty_cache()
+
+    # ---- prefill M = 2048 (two weight copies alternate: 224 MB > L2); after
+    # the memory-bound sections, whose numbers a power-capped tensor-core
+    # loop just before would skew
+    def prefill_round():
+        for c in copies[:2]:
+            w8.linear(Xp, c, scales, out=Yp)
+
+    g_pf = capture(prefill_round, stream)
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            g_pf.replay()
+    torch.cuda.synchronize()
+    n_pf = max(5, args.prefill_reps)
+    t_pf = timed_replays(g_pf, n_pf, stream, ws, device, sampler)
+    pf_window = sampler.windows[-1]
+    pf_s = t_pf / (2 * n_pf)
+    pf_flops = 2.0 * M_PREFILL * K_DIM * N_DIM
+    pf_tflops = pf_flops / pf_s / 1e12
+    pf_peak, pf_peak_name = tensor_peak(t_pf, tf_peak, tf_sustained)
+    pf_med_s = statistics.median(replay_times(g_pf, 50, stream, ws, device, sampler)) / 2
+
+    # ---- the variants' prefill calls (M = 2048), each timed as the plain
+    # call is (a graph of two calls, back to back), with the plain call timed
+    # again just before them so that the ratios compare like with like
+    if not args.no_variants:
+        fl_pf = 2.0 * M_PREFILL * K_DIM * N_DIM
+        t_plain = graph_time(lambda: [w8.linear(Xp, c, scales, out=Yp) for c in copies[:2]], 20) / 2
+        t_pa = graph_time(lambda: [w8.linear_asym(Xp, c, sa, za, out=Yp) for c in pa], 20) / 2
+        t_po = graph_time(lambda: [w8.linear_outliers(Xp, c, so, co, ro, vo, out=Yp) for c in po], 20) / 2
+        variants["asymmetric"].update({
+            "prefill_m2048_us": round(t_pa * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_pa / 1e12, 1),
+            "prefill_m2048_frac_tensor_burst": round(fl_pf / t_pa / 1e12 / tf_peak, 4),
+            "prefill_m2048_vs_plain": round(t_pa / t_plain, 3)})
+        variants["outlier_split"].update({
             "prefill_m2048_us": round(t_po * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_po / 1e12, 1),
             "prefill_m2048_frac_tensor_burst": round(fl_pf / t_po / 1e12 / tf_peak, 4),
-            "prefill_m2048_vs_plain": round(t_po / pf_med_s, 3)}
-        del po, qo, qc
+            "prefill_m2048_vs_plain": round(t_po / t_plain, 3)})
+        variants["prefill_m2048_plain_us_alongside"] = round(t_plain * 1e6, 1)
+        del pa, po
         torch.cuda.empty_cache()
 
     # ---- the prefill sweep: M in {512, 1024, 2048} on 4096 x 27392 and
@@ -720,8 +736,8 @@ def run_native(args, ws, rank, local):
 # ------------------------------------------------------------------ profiling driver
 def run_profile(args):
     """A few plain launches of one kernel, for ncu captures (no graphs, no
-    timing): the bench's workload, or the weight shape --profile-shape KxN.
-    Packed-weight copies alternate (at least 2, and enough for more than
+    timing): the bench's workload, or the weight shape --profile-shape KxN
+    (and --profile-m tokens).  Packed-weight copies alternate (at least 2, and enough for more than
     256 MB), so the weight is not served from L2."""
     import torch
     import synthetic
@@ -739,6 +755,8 @@ def run_profile(args):
     ncp = max(2, -(-(256 << 20) // (K * N)))
     copies = [w8.prepack(q) for _ in range(ncp)]
     M = {"decode": M_DECODE, "decode16": 16, "prefill": M_PREFILL}.get(args.profile, M_DECODE)
+    if args.profile_m:
+        M = args.profile_m
     X = torch.from_numpy(synthetic.activations(M, K, synthetic.SEED, tid + 1)).to(device)
     Y = torch.empty((M, N), dtype=torch.float16, device=device)
     torch.cuda.synchronize()
@@ -747,6 +765,8 @@ def run_profile(args):
             w8.linear(X, copies[i % ncp], scales, out=Y)
         elif args.profile == "quantize":
             w8.quantize(W, q=q, scales=scales)
+        elif args.profile == "percentile":
+            w8.quantize_clip(W, "percentile", 0.999, q=q, scales=scales)
         elif args.profile == "prepack":
             w8.prepack(q, out=copies[i % ncp])
     torch.cuda.synchronize()
@@ -967,10 +987,12 @@ def main():
     ap.add_argument("--set-reps", type=int, default=100)
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the variant, prefill-sweep and BERT sections")
-    ap.add_argument("--profile", choices=["decode", "decode16", "prefill", "quantize", "prepack"],
+    ap.add_argument("--profile", choices=["decode", "decode16", "prefill", "quantize", "percentile", "prepack"],
                     help="run --steps plain launches of one kernel (for ncu) and exit")
     ap.add_argument("--profile-shape", default="",
                     help="weight shape KxN for --profile (default: the bench's 4096x27392)")
+    ap.add_argument("--profile-m", type=int, default=0,
+                    help="tokens M for a linear --profile (default: the profile's own)")
     args = ap.parse_args()
     if args.profile:
         return run_profile(args)

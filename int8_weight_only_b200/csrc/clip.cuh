@@ -6,17 +6,32 @@
 //   s_n = fp16_rne( fp32(bound_n) / 127 ),  q = clamp( rne(W / s_n), -127, 127 ).
 //
 // The order statistic is found by radix selection on the bit pattern of
-// |w| (for non-negative floats the pattern orders as the value): four
-// passes over the channel, each a 256-bin histogram of one byte of the
-// pattern among the values whose higher bytes equal those already chosen;
-// the bin holding the t-th largest fixes that byte.  A fifth pass writes
-// the codes.
+// |w| (for non-negative floats the pattern orders as the value, and the
+// sign bit is clear, so a pattern has 31 bits).  A column's selection goes
+// digit by digit from the top -- a 10-bit digit first, then 7-bit ones --
+// keeping the prefix of the bound's pattern found so far and the rank
+// still to find among the values that carry that prefix.  A pass over the
+// column does one of two things for it:
+//  - histogram: count the values with the prefix by their next digit; the
+//    bin that holds the wanted rank extends the prefix;
+//  - collect: once at most kCap values carry the prefix, copy their
+//    patterns into shared memory, and finish the selection there (digit
+//    by digit again, within one warp, with no further pass over W).
+// On the usual weights the first pass (10-bit histogram) leaves a few
+// values in the chosen bin, the second collects them and the third writes
+// the codes: three passes over W instead of the five a byte-wise radix
+// select takes.  A column whose values crowd into one bin at every digit
+// (all equal, say) takes at most four selection passes.
 //
 // Work unit: a panel of 32 columns over all K rows, one CTA per panel
 // (persistent CTAs walk the panels).  A producer thread streams the panel
-// five times through a ring of 2-D TMA boxes (32 columns x 16 KB of rows);
-// pass 1 loads keep the panel in L2 (evict-last) for the four passes that
-// follow.  Consumer lane = column: each warp takes every 16th row of a box.
+// once per pass through a ring of 2-D TMA boxes (32 columns x 16 KB of
+// rows) with the L2 evict-last hint, so that passes after the first read
+// L2.  How many passes a panel takes is known only once its columns are
+// resolved, so before each pass after the second the producer waits for
+// the consumers' verdict on the pass two before it (the panel needs pass j
+// exactly when pass j - 1 is still a selection pass).  Consumer lane =
+// column: each warp takes every 16th row of a box.
 #pragma once
 
 #include "common.cuh"
@@ -29,12 +44,22 @@ constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr int kPanel = 32;
-constexpr int kStages = 8;
+constexpr int kStages = 5;
 constexpr int kBoxBytes = 16384;
-constexpr int kBins = 256;
-constexpr int kBinStride = kBins + 1;   // per-column rows offset by one bank
-constexpr int kPasses = 5;              // four selection passes, then the codes
-constexpr int kSmemBytes = kStages * kBoxBytes + 1024;
+constexpr int kCap = 1024;               // values a column collects; bins of the first digit
+constexpr int kRegion = kCap + 1;        // words per column (rows offset by one bank)
+constexpr int kRegionBytes = kPanel * kRegion * 4;
+constexpr int kScratch = 128;            // words of a warp's histogram in a collected column's selection
+constexpr int kSmemBytes = kStages * kBoxBytes + 1024 + kRegionBytes + kConsumerWarps * kScratch * 4;
+constexpr unsigned SITE_CLIP_DECIDE = 0x53;   // producer: the consumers' verdict on a pass
+
+// Column modes of a selection pass.
+constexpr int kDone = 0, kHist = 1, kCollect = 2;
+
+// Width of the digit after `lvl` resolved top bits: 10 first, then 7.
+__host__ __device__ constexpr int digit_width(int lvl) { return lvl == 0 ? 10 : (31 - lvl < 7 ? 31 - lvl : 7); }
+// Mask of the top `lvl` bits of a 31-bit pattern.
+__device__ __forceinline__ uint32_t prefix_mask(int lvl) { return lvl == 0 ? 0u : ~((1u << (31 - lvl)) - 1u); }
 
 template <typename T>
 struct Geo {
@@ -75,6 +100,135 @@ __device__ __forceinline__ float load_elem<__half>(const uint8_t *p) {
     return __half2float(*reinterpret_cast<const __half *>(p));
 }
 
+// One warp: the bin of histogram hb[0, nb) (bins ordered by value, nb a
+// power of two from 8 to 1024) that holds the rem-th largest of the counted
+// values.  rem becomes the rank within that bin and grp the bin's count.
+// Lane l sums bins [l cs, l cs + cs), cs = max(1, nb / 32) (the 32-bin
+// chunks read in a rotated order, so the lanes hit distinct banks); the
+// suffix sums over the lanes locate the chunk, and a second suffix scan
+// within the chunk the bin.
+__device__ __forceinline__ int select_bin(const uint32_t *hb, int nb, int lane, uint32_t &rem, uint32_t &grp) {
+    const int cs = nb >= 32 ? nb / 32 : 1;
+    uint32_t sum = 0;
+    if (cs == 32) {
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) sum += hb[lane * 32 + ((i + lane) & 31)];
+    } else {
+        for (int i = 0; i < cs; ++i) {
+            const int b = lane * cs + i;
+            if (b < nb) sum += hb[b];
+        }
+    }
+    uint32_t s = sum;   // values in the chunks of this lane and above
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, s, off);
+        if (lane + off < 32) s += y;
+    }
+    const uint32_t ball = __ballot_sync(0xffffffffu, s >= rem);
+    const int lc = ball ? 31 - __clz(ball) : 0;   // the total is at least rem: lane 0 is set
+    const uint32_t above = __shfl_sync(0xffffffffu, s - sum, lc);
+    const int b0 = lc * cs;
+    const uint32_t h = (lane < cs && b0 + lane < nb) ? hb[b0 + lane] : 0u;
+    uint32_t s2 = h;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, s2, off);
+        if (lane + off < 32) s2 += y;
+    }
+    const uint32_t ball2 = __ballot_sync(0xffffffffu, lane < cs && above + s2 >= rem);
+    const int lb = ball2 ? 31 - __clz(ball2) : 0;
+    const uint32_t above_b = above + __shfl_sync(0xffffffffu, s2 - h, lb);
+    grp = __shfl_sync(0xffffffffu, h, lb);
+    rem -= above_b;
+    return b0 + lb;
+}
+
+// What a pass does with a warp's rows of one box (lane = column):
+//  kScanHist0     first pass, K > kCap: count every value by its 10-bit digit
+//  kScanCollect0  first pass, K <= kCap: keep every pattern (slot = row)
+//  kScanSelect    later selection passes, each column by its own mode
+//  kScanCode      the code pass
+// kCheck: the box holds rows past K (only the last one can).
+constexpr int kScanHist0 = 0, kScanCollect0 = 1, kScanSelect = 2, kScanCode = 3;
+
+struct LaneScan {
+    uint32_t mask, prefix, dmask;   // selection: the column's prefix test and digit
+    int shift;
+    bool hist;                      // selection: histogram (else collect)
+    float sc, inv;                  // code pass: the scale and fl(1 / scale)
+    uint32_t bound;                 // code pass: the bound's pattern
+    bool n_ok;                      // the column is inside the weight
+};
+
+template <typename T, int kKind, bool kCheck, bool kOut>
+__device__ __forceinline__ void scan_box(const uint8_t *box, int k0, int K, int warp, int lane, const LaneScan &ls,
+                                         uint32_t *hb, int *cnt, int *on, int8_t *qcol, int64_t N) {
+    using G = Geo<T>;
+    constexpr int kPer = G::kRows / kConsumerWarps;
+    // the warp's rows, loaded before any shared memory update (atomics and
+    // stores to the same memory would otherwise order every load after the
+    // last update)
+    float vals[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u)
+        vals[u] = load_elem<T>(box + (warp + u * kConsumerWarps) * G::kRowBytes + lane * (int)sizeof(T));
+    if constexpr (kKind == kScanCode) {
+        if (!ls.n_ok) return;
+        // one decision for the warp's rows: the fast codes, or the
+        // quotient's where any of them is near a rounding boundary
+        int code[kPer];
+        bool sure = true;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            bool su;
+            code[u] = quant::quantize_fast(vals[u], ls.inv, su);
+            sure &= su;
+        }
+        if (!sure) {
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) code[u] = quant::quantize_exact(vals[u], ls.sc);
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int k = k0 + warp + u * kConsumerWarps;
+            if (kCheck && k >= K) break;
+            if constexpr (kOut) {
+                if (abs_bits(vals[u]) > ls.bound) {   // |w| above the bound
+                    const int j = atomicAdd(on, 1);
+                    if (j < kMaxOutliers) {
+                        reinterpret_cast<int32_t *>(hb)[j] = k;
+                        reinterpret_cast<uint16_t *>(hb + kMaxOutliers)[j] = __half_as_ushort(__float2half_rn(vals[u]));
+                    }
+                    code[u] = 0;
+                }
+            }
+            qcol[(int64_t)k * N] = (int8_t)code[u];
+        }
+    } else {
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int k = k0 + warp + u * kConsumerWarps;
+            if (kCheck && k >= K) break;
+            const uint32_t bits = abs_bits(vals[u]);
+            if constexpr (kKind == kScanHist0) {
+                atomicAdd(&hb[bits >> 21], 1u);
+            } else if constexpr (kKind == kScanCollect0) {
+                hb[k] = bits;
+            } else {
+                if ((bits & ls.mask) == ls.prefix) {
+                    if (ls.hist) {
+                        atomicAdd(&hb[(bits >> ls.shift) & ls.dmask], 1u);
+                    } else {
+                        const int j = atomicAdd(cnt, 1);
+                        if (j < kCap) hb[j] = bits;
+                    }
+                }
+            }
+        }
+    }
+}
+
 // grid = persistent CTAs, kThreads threads, kSmemBytes dynamic shared
 // memory.  tmap_w: W [K, N], box 32 columns x Geo<T>::kRows rows, no swizzle.
 template <typename T, bool kOut>
@@ -84,25 +238,34 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
     extern __shared__ uint8_t smem_raw[];
     uint8_t *ring = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // per column: the histogram or the collected patterns of a selection
+    // pass; the outlier lists during the code pass
+    uint32_t *region = reinterpret_cast<uint32_t *>(ring + kStages * kBoxBytes);
+    uint32_t *scratch = region + kPanel * kRegion;
     __shared__ uint64_t full[kStages], empty[kStages];
-    __shared__ uint32_t hist[kPanel * kBinStride];
-    __shared__ uint32_t col_prefix[kPanel];   // chosen high bytes of the bound's pattern
-    __shared__ int col_rem[kPanel];           // rank still to find within them
+    __shared__ uint64_t decide[2];            // the verdicts, alternating
+    __shared__ int verdict[2];                // 1: the pass after the next one is needed
+    __shared__ uint32_t col_prefix[kPanel];   // top bits of the bound's pattern found so far
+    __shared__ int col_lvl[kPanel];           // how many of its 31 bits
+    __shared__ uint32_t col_rem[kPanel];      // rank still to find among the values with the prefix
+    __shared__ uint32_t col_grp[kPanel];      // how many values carry the prefix
+    __shared__ int col_mode[kPanel];
+    __shared__ int col_cnt[kPanel];           // collected so far
     __shared__ float col_scale[kPanel], col_inv[kPanel];
-    // outlier split: this panel's side lists, filled in the code pass
-    __shared__ int o_n[kOut ? kPanel : 1];
-    __shared__ int32_t o_row[kOut ? kPanel : 1][kOut ? kMaxOutliers : 1];
-    __shared__ uint16_t o_val[kOut ? kPanel : 1][kOut ? kMaxOutliers : 1];
+    __shared__ int o_n[kPanel];               // outlier split: listed so far
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int nbox = (int)((p.K + G::kRows - 1) / G::kRows);
+    const int K = (int)p.K;
+    const int nbox = (K + G::kRows - 1) / G::kRows;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kConsumerWarps);
         }
+        mbar_init(&decide[0], 1);
+        mbar_init(&decide[1], 1);
         fence_barrier_init();
         prefetch_tensormap(&tmap_w);
     }
@@ -111,18 +274,25 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+            const uint64_t keep = policy_evict_last();
             int s = 0;
             uint32_t ph = 0;
             int issued = 0;
+            uint32_t nd = 0;   // verdicts read
             bool ok = true;
             for (int panel = blockIdx.x; panel < p.panels && ok; panel += gridDim.x) {
-                for (int pass = 0; pass < kPasses && ok; ++pass) {
+                for (int pass = 0; ok; ++pass) {
+                    if (pass >= 2) {
+                        // pass `pass` exists when pass - 1 is a selection pass
+                        if (!mbar_wait_parked(&decide[nd & 1], (nd >> 1) & 1, SITE_CLIP_DECIDE)) { ok = false; break; }
+                        const int more = *reinterpret_cast<volatile int *>(&verdict[nd & 1]);
+                        ++nd;
+                        if (!more) break;
+                    }
                     for (int i = 0; i < nbox; ++i) {
                         if (!mbar_wait_parked(&empty[s], ph ^ 1u, SITE_CLIP_EMPTY)) { ok = false; break; }
                         mbar_arrive_expect_tx(&full[s], kBoxBytes);
-                        tma_load_2d_hint(ring + s * kBoxBytes, &tmap_w, panel * kPanel, i * G::kRows, &full[s],
-                                         pass + 1 < kPasses ? keep : drop);
+                        tma_load_2d_hint(ring + s * kBoxBytes, &tmap_w, panel * kPanel, i * G::kRows, &full[s], keep);
                         ++issued;
                         if (++s == kStages) { s = 0; ph ^= 1u; }
                     }
@@ -143,60 +313,77 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
     const int c = threadIdx.x;
     int s = 0;
     uint32_t ph = 0;
+    uint32_t nd = 0;   // verdicts given
     bool ok = true;
     for (int panel = blockIdx.x; panel < p.panels && ok; panel += gridDim.x) {
         if (c < kPanel) {
+            const bool in = (int64_t)panel * kPanel + c < p.N;
             col_prefix[c] = 0;
-            col_rem[c] = p.t;
-            if constexpr (kOut) o_n[c] = 0;
+            col_lvl[c] = 0;
+            col_rem[c] = (uint32_t)p.t;
+            col_grp[c] = (uint32_t)K;
+            col_mode[c] = !in ? kDone : (K <= kCap ? kCollect : kHist);
+            col_cnt[c] = K <= kCap ? K : 0;   // the first pass keeps every row's pattern, in slot = row
         }
-        for (int i = c; i < kPanel * kBinStride; i += kConsumers) hist[i] = 0;
-        for (int pass = 0; pass < kPasses; ++pass) {
-            // the histogram is zero and the column state of the last scan
-            // is visible
+        bool code_pass = false;
+        for (int pass = 0; ok; ++pass) {
+            // the column state of the last resolution is visible
             if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
-            const int shift = 24 - 8 * pass;   // byte of the pattern this pass histograms
-            const uint32_t hi_mask = pass == 0 ? 0u : ~((1u << (shift + 8)) - 1u);
-            // pass 4: col_prefix holds the bound's pattern
-            const uint32_t prefix = col_prefix[lane];
-            const float sc = pass == 4 ? col_scale[lane] : 0.0f;
-            const float inv = pass == 4 ? col_inv[lane] : 0.0f;
-            const int64_t n = (int64_t)panel * kPanel + lane;
+            const int mode = col_mode[lane];
+            if (!code_pass) {
+                // clear the histograms of this pass: warp w, columns w and w + 16
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int col = warp + h * kConsumerWarps;
+                    if (col_mode[col] == kHist) {
+                        const int nb = 1 << digit_width(col_lvl[col]);
+                        for (int b = lane; b < nb; b += 32) region[col * kRegion + b] = 0u;
+                    }
+                }
+                if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
+            }
+            // this lane's column: what to match and where to count it
+            LaneScan ls;
+            {
+                const int lvl = col_lvl[lane];
+                ls.mask = mode == kDone ? 0u : prefix_mask(lvl);
+                ls.prefix = mode == kDone ? 0xFFFFFFFFu : col_prefix[lane];   // no pattern matches
+                ls.shift = 31 - lvl - digit_width(lvl);
+                ls.dmask = (1u << digit_width(lvl)) - 1u;
+                ls.hist = mode == kHist;
+                ls.sc = code_pass ? col_scale[lane] : 0.0f;
+                ls.inv = code_pass ? col_inv[lane] : 0.0f;
+                ls.bound = col_prefix[lane];
+                ls.n_ok = (int64_t)panel * kPanel + lane < p.N;
+            }
+            uint32_t *const hb = region + lane * kRegion;
+            int8_t *const qcol = p.q + (int64_t)panel * kPanel + lane;
+            // which form this pass takes (the same in every warp)
+            const int kind = code_pass ? kScanCode : (pass > 0 ? kScanSelect : (K > kCap ? kScanHist0 : kScanCollect0));
             for (int i = 0; i < nbox; ++i) {
                 if (ok && !warp_all(mbar_wait_parked(&full[s], ph, SITE_CLIP_LOAD))) ok = false;
                 if (ok) {
                     const uint8_t *box = ring + s * kBoxBytes;
-                    for (int rloc = warp; rloc < G::kRows; rloc += kConsumerWarps) {
-                        const int64_t k = (int64_t)i * G::kRows + rloc;
-                        if (k >= p.K) break;
-                        const float v = load_elem<T>(box + rloc * G::kRowBytes + lane * (int)sizeof(T));
-                        if (pass < 4) {
-                            const uint32_t bits = abs_bits(v);
-                            if ((bits & hi_mask) == prefix)
-                                atomicAdd(&hist[lane * kBinStride + ((bits >> shift) & 0xFFu)], 1u);
-                        } else if (n < p.N) {
-                            bool sure;
-                            int code = quant::quantize_fast(v, inv, sure);
-                            if (!sure) code = quant::quantize_exact(v, sc);
-                            if constexpr (kOut) {
-                                if (abs_bits(v) > prefix) {   // |w| above the bound
-                                    const int j = atomicAdd(&o_n[lane], 1);
-                                    if (j < kMaxOutliers) {
-                                        o_row[lane][j] = (int32_t)k;
-                                        o_val[lane][j] = __half_as_ushort(__float2half_rn(v));
-                                    }
-                                    code = 0;
-                                }
-                            }
-                            p.q[k * p.N + n] = (int8_t)code;
-                        }
-                    }
+                    const int k0 = i * G::kRows;
+                    const bool chk = k0 + G::kRows > K;
+#define W8_SCAN(KIND)                                                                                       \
+    (chk ? scan_box<T, KIND, true, kOut>(box, k0, K, warp, lane, ls, hb, &col_cnt[lane], &o_n[lane], qcol, p.N) \
+         : scan_box<T, KIND, false, kOut>(box, k0, K, warp, lane, ls, hb, &col_cnt[lane], &o_n[lane], qcol, p.N))
+                    if (kind == kScanCode)
+                        W8_SCAN(kScanCode);
+                    else if (kind == kScanSelect)
+                        W8_SCAN(kScanSelect);
+                    else if (kind == kScanHist0)
+                        W8_SCAN(kScanHist0);
+                    else
+                        W8_SCAN(kScanCollect0);
+#undef W8_SCAN
                 }
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(&empty[s]);
                 if (++s == kStages) { s = 0; ph ^= 1u; }
             }
-            if (pass == 4) {
+            if (code_pass) {
                 if constexpr (kOut) {
                     // every outlier of the panel is listed: sort each column's
                     // list by row (the order the warps met them varies) and
@@ -204,57 +391,103 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
                     if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
                     const int64_t nn = (int64_t)panel * kPanel + c;
                     if (c < kPanel && nn < p.N) {
+                        int32_t *orow = reinterpret_cast<int32_t *>(region + c * kRegion);
+                        uint16_t *oval = reinterpret_cast<uint16_t *>(region + c * kRegion + kMaxOutliers);
                         const int cnt = min(o_n[c], p.cap);
                         for (int a = 1; a < cnt; ++a) {
-                            const int32_t r0 = o_row[c][a];
-                            const uint16_t v0 = o_val[c][a];
+                            const int32_t r0 = orow[a];
+                            const uint16_t v0 = oval[a];
                             int b2 = a - 1;
-                            for (; b2 >= 0 && o_row[c][b2] > r0; --b2) {
-                                o_row[c][b2 + 1] = o_row[c][b2];
-                                o_val[c][b2 + 1] = o_val[c][b2];
+                            for (; b2 >= 0 && orow[b2] > r0; --b2) {
+                                orow[b2 + 1] = orow[b2];
+                                oval[b2 + 1] = oval[b2];
                             }
-                            o_row[c][b2 + 1] = r0;
-                            o_val[c][b2 + 1] = v0;
+                            orow[b2 + 1] = r0;
+                            oval[b2 + 1] = v0;
                         }
                         p.o_count[nn] = cnt;
                         for (int j = 0; j < p.cap; ++j) {
-                            p.o_rows[nn * p.cap + j] = j < cnt ? o_row[c][j] : 0;
-                            p.o_vals[nn * p.cap + j] = j < cnt ? o_val[c][j] : (uint16_t)0;
+                            p.o_rows[nn * p.cap + j] = j < cnt ? orow[j] : 0;
+                            p.o_vals[nn * p.cap + j] = j < cnt ? oval[j] : (uint16_t)0;
                         }
                     }
-                    // the lists are read before the next panel resets them
-                    if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
                 }
+                // the next panel's state is written after every read of this one
+                if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
                 break;
             }
-            // the histogram is complete
+            // ------------------------------------------------ resolution
+            // every count and pattern of the pass is in shared memory
             if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
-            if (c < kPanel) {
-                // the bin that holds the rem-th largest of the matching values
-                const int rem = col_rem[c];
-                uint32_t cum = 0;
-                int b = kBins - 1;
-                for (; b > 0; --b) {
-                    const uint32_t h = hist[c * kBinStride + b];
-                    if (cum + h >= (uint32_t)rem) break;
-                    cum += h;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                const int col = warp + h * kConsumerWarps;
+                const int cmode = col_mode[col];
+                if (cmode == kDone) continue;
+                uint32_t *const cb = region + col * kRegion;
+                int clvl = col_lvl[col];
+                uint32_t pre = col_prefix[col];
+                uint32_t rem = col_rem[col];
+                uint32_t grp = col_grp[col];
+                int nmode;
+                if (cmode == kHist) {
+                    const int w = digit_width(clvl);
+                    const int b = select_bin(cb, 1 << w, lane, rem, grp);
+                    pre |= (uint32_t)b << (31 - clvl - w);
+                    clvl += w;
+                    nmode = clvl == 31 ? kDone : (grp <= (uint32_t)kCap ? kCollect : kHist);
+                } else {
+                    // the collected patterns stay where they are; each digit's
+                    // histogram goes to the warp's scratch
+                    const int cnt = min(col_cnt[col], kCap);
+                    uint32_t *const sb = scratch + warp * kScratch;
+#pragma unroll 1
+                    while (clvl < 31) {
+                        const int w = digit_width(clvl == 0 ? 1 : clvl);   // 7-bit digits here
+                        const int sh = 31 - clvl - w;
+                        const uint32_t m = prefix_mask(clvl);
+                        for (int b = lane; b < (1 << w); b += 32) sb[b] = 0u;
+                        __syncwarp();
+                        for (int j = lane; j < cnt; j += 32) {
+                            const uint32_t x = cb[j];
+                            if ((x & m) == pre) atomicAdd(&sb[(x >> sh) & ((1u << w) - 1u)], 1u);
+                        }
+                        __syncwarp();
+                        const int b = select_bin(sb, 1 << w, lane, rem, grp);
+                        pre |= (uint32_t)b << sh;
+                        clvl += w;
+                        __syncwarp();
+                    }
+                    nmode = kDone;
                 }
-                col_rem[c] = rem - (int)cum;
-                const uint32_t pre = col_prefix[c] | ((uint32_t)b << shift);
-                col_prefix[c] = pre;
-                if (pass == 3) {
-                    const float bound = __uint_as_float(pre);
-                    const __half s16 = __float2half_rn(__fdiv_rn(bound, 127.0f));
-                    const float sf = __half2float(s16);
-                    col_scale[c] = sf;
-                    col_inv[c] = sf != 0.0f ? __frcp_rn(sf) : 0.0f;
-                    const int64_t nn = (int64_t)panel * kPanel + c;
-                    if (nn < p.N) p.scales[nn] = __half_as_ushort(s16);
+                if (lane == 0) {
+                    col_prefix[col] = pre;
+                    col_lvl[col] = clvl;
+                    col_rem[col] = rem;
+                    col_grp[col] = grp;
+                    col_mode[col] = nmode;
+                    col_cnt[col] = 0;
                 }
             }
-            // the scan has read the histogram: clear it for the next pass
             if (!named_bar_all(1, kConsumers, ok)) { ok = false; break; }
-            for (int i = c; i < kPanel * kBinStride; i += kConsumers) hist[i] = 0;
+            code_pass = __all_sync(0xffffffffu, col_mode[lane] == kDone);
+            if (c == 0) {
+                // the producer loads the pass after the next one only if the
+                // next one selects
+                verdict[nd & 1] = code_pass ? 0 : 1;
+                mbar_arrive(&decide[nd & 1]);
+            }
+            ++nd;
+            if (code_pass && c < kPanel) {
+                const float bound = __uint_as_float(col_prefix[c]);
+                const __half s16 = __float2half_rn(__fdiv_rn(bound, 127.0f));
+                const float sf = __half2float(s16);
+                col_scale[c] = sf;
+                col_inv[c] = sf != 0.0f ? __frcp_rn(sf) : 0.0f;
+                o_n[c] = 0;
+                const int64_t nn = (int64_t)panel * kPanel + c;
+                if (nn < p.N) p.scales[nn] = __half_as_ushort(s16);
+            }
         }
     }
 }

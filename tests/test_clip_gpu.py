@@ -9,7 +9,7 @@ from tests.gpu_helpers import SEED, assert_close, to_gpu, to_np, w8
 
 pytestmark = pytest.mark.gpu
 
-SHAPES = [(64, 8), (256, 512), (1000, 264), (4096, 4608), (13696, 128)]
+SHAPES = [(64, 8), (256, 512), (1000, 264), (1024, 40), (1025, 40), (4096, 4608), (13696, 128)]
 
 
 def _check(W, mode, param):
@@ -44,6 +44,25 @@ def test_percentile_with_ties_and_zero_columns():
     W[:, 8] = 0.5
     for p in (0.9, 0.5, 0.99, 1.0):
         _check(W, "percentile", p)
+
+
+def test_percentile_crowded_leading_digits():
+    # Half of each column's rows share their leading bits in large numbers:
+    # 3000 values 0.5 (1 + m 2^-23) with m below 2^21, 2^10 or 2^3 carry one
+    # leading 10-bit digit (more than a column can collect at once), and
+    # with the smaller ranges also one or two further 7-bit digits, so the
+    # selection goes on histogramming before it collects, or never collects.
+    rng = np.random.default_rng(37)
+    K, N = 6000, 72
+    W = rng.normal(0.0, 0.02, size=(K, N)).astype(np.float32)
+    for lo, hi, bits in ((0, 16, 21), (16, 32, 10), (48, 72, 3)):
+        rows = rng.permutation(K)[:3000]
+        m = rng.integers(0, 1 << bits, size=(3000, hi - lo))
+        sign = np.where(rng.random((3000, hi - lo)) < 0.5, -1.0, 1.0)
+        W[rows, lo:hi] = (sign * 0.5 * (1.0 + m * 2.0 ** -23)).astype(np.float32)
+    for p in (0.9, 0.5, 0.25, 0.999, 1e-4):
+        _check(W, "percentile", p)
+    _check(W.astype(np.float16), "percentile", 0.5)
 
 
 def test_percentile_matches_plain_quantizer_at_p_one():
