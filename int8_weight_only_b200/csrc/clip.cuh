@@ -8,16 +8,16 @@
 // The order statistic is found by radix selection on the bit pattern of
 // |w| (for non-negative floats the pattern orders as the value, and the
 // sign bit is clear, so a pattern has 31 bits).  A column's selection goes
-// digit by digit from the top -- a 10-bit digit first, then 7-bit ones --
-// keeping the prefix of the bound's pattern found so far and the rank
-// still to find among the values that carry that prefix.  A pass over the
-// column does one of two things for it:
+// digit by digit from the top -- digits of 9, 8, 7 and 7 bits -- keeping
+// the prefix of the bound's pattern found so far and the rank still to
+// find among the values that carry that prefix.  A pass over the column
+// does one of two things for it:
 //  - histogram: count the values with the prefix by their next digit; the
 //    bin that holds the wanted rank extends the prefix;
 //  - collect: once at most kCap values carry the prefix, copy their
 //    patterns into shared memory, and finish the selection there (digit
 //    by digit again, within one warp, with no further pass over W).
-// On the usual weights the first pass (10-bit histogram) leaves a few
+// On the usual weights the first pass (a 512-bin histogram) leaves a few
 // values in the chosen bin, the second collects them and the third writes
 // the codes: three passes over W instead of the five a byte-wise radix
 // select takes.  A column whose values crowd into one bin at every digit
@@ -30,8 +30,10 @@
 // L2.  How many passes a panel takes is known only once its columns are
 // resolved, so before each pass after the second the producer waits for
 // the consumers' verdict on the pass two before it (the panel needs pass j
-// exactly when pass j - 1 is still a selection pass).  Consumer lane =
-// column: each warp takes every 16th row of a box.
+// exactly when pass j - 1 is still a selection pass).  In the selection
+// passes consumer lane = column and each warp takes every 16th row of a
+// box; the code pass uses the plain quantizer's layout (a thread per
+// 16-byte row segment).
 #pragma once
 
 #include "common.cuh"
@@ -44,9 +46,10 @@ constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr int kPanel = 32;
-constexpr int kStages = 5;
+constexpr int kStages = 7;
 constexpr int kBoxBytes = 16384;
-constexpr int kCap = 1024;               // values a column collects; bins of the first digit
+constexpr int kCap = 768;                // values a column collects
+constexpr int kFirstBits = 9;            // width of the first digit (512 bins)
 constexpr int kRegion = kCap + 1;        // words per column (rows offset by one bank)
 constexpr int kRegionBytes = kPanel * kRegion * 4;
 constexpr int kScratch = 128;            // words of a warp's histogram in a collected column's selection
@@ -57,7 +60,11 @@ constexpr unsigned SITE_CLIP_DECIDE = 0x53;   // producer: the consumers' verdic
 constexpr int kDone = 0, kHist = 1, kCollect = 2;
 
 // Width of the digit after `lvl` resolved top bits: 10 first, then 7.
-__host__ __device__ constexpr int digit_width(int lvl) { return lvl == 0 ? 10 : (31 - lvl < 7 ? 31 - lvl : 7); }
+__host__ __device__ constexpr int digit_width(int lvl) {
+    return lvl == 0 ? kFirstBits : (lvl == kFirstBits ? 8 : (31 - lvl < 7 ? 31 - lvl : 7));
+}
+// Width of a digit in a collected column's selection (its histogram is a warp's 128-word scratch).
+__host__ __device__ constexpr int collect_width(int lvl) { return 31 - lvl < 7 ? 31 - lvl : 7; }
 // Mask of the top `lvl` bits of a 31-bit pattern.
 __device__ __forceinline__ uint32_t prefix_mask(int lvl) { return lvl == 0 ? 0u : ~((1u << (31 - lvl)) - 1u); }
 
@@ -89,6 +96,17 @@ struct Params {
 
 __device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
 
+// Shared-memory atomics named as such (the histogram and the lists live in
+// a dynamic shared-memory region the compiler would address generically).
+__device__ __forceinline__ void red_add_shared(uint32_t *p, uint32_t v) {
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v));
+}
+__device__ __forceinline__ int atom_add_shared(int *p, int v) {
+    int r;
+    asm volatile("atom.shared.add.u32 %0, [%1], %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(v));
+    return r;
+}
+
 template <typename T>
 __device__ __forceinline__ float load_elem(const uint8_t *p);
 template <>
@@ -110,14 +128,11 @@ __device__ __forceinline__ float load_elem<__half>(const uint8_t *p) {
 __device__ __forceinline__ int select_bin(const uint32_t *hb, int nb, int lane, uint32_t &rem, uint32_t &grp) {
     const int cs = nb >= 32 ? nb / 32 : 1;
     uint32_t sum = 0;
-    if (cs == 32) {
-#pragma unroll 8
-        for (int i = 0; i < 32; ++i) sum += hb[lane * 32 + ((i + lane) & 31)];
-    } else {
-        for (int i = 0; i < cs; ++i) {
-            const int b = lane * cs + i;
-            if (b < nb) sum += hb[b];
-        }
+    if (nb >= 32) {
+#pragma unroll 4
+        for (int i = 0; i < cs; ++i) sum += hb[lane * cs + ((i + lane) & (cs - 1))];
+    } else if (lane < nb) {
+        sum = hb[lane];
     }
     uint32_t s = sum;   // values in the chunks of this lane and above
 #pragma unroll
@@ -144,26 +159,23 @@ __device__ __forceinline__ int select_bin(const uint32_t *hb, int nb, int lane, 
     return b0 + lb;
 }
 
-// What a pass does with a warp's rows of one box (lane = column):
-//  kScanHist0     first pass, K > kCap: count every value by its 10-bit digit
+// What a selection pass does with a warp's rows of one box (lane = column):
+//  kScanHist0     first pass, K > kCap: count every value by its first digit
 //  kScanCollect0  first pass, K <= kCap: keep every pattern (slot = row)
-//  kScanSelect    later selection passes, each column by its own mode
-//  kScanCode      the code pass
-// kCheck: the box holds rows past K (only the last one can).
+//  kScanSelect    later passes, each column by its own mode
+// (kScanCode, the code pass, is code_box below.)  kCheck: the box holds
+// rows past K (only the last one can).
 constexpr int kScanHist0 = 0, kScanCollect0 = 1, kScanSelect = 2, kScanCode = 3;
 
 struct LaneScan {
-    uint32_t mask, prefix, dmask;   // selection: the column's prefix test and digit
+    uint32_t mask, prefix, dmask;   // the column's prefix test and digit
     int shift;
-    bool hist;                      // selection: histogram (else collect)
-    float sc, inv;                  // code pass: the scale and fl(1 / scale)
-    uint32_t bound;                 // code pass: the bound's pattern
-    bool n_ok;                      // the column is inside the weight
+    bool hist;                      // histogram (else collect)
 };
 
 template <typename T, int kKind, bool kCheck, bool kOut>
 __device__ __forceinline__ void scan_box(const uint8_t *box, int k0, int K, int warp, int lane, const LaneScan &ls,
-                                         uint32_t *hb, int *cnt, int *on, int8_t *qcol, int64_t N) {
+                                         uint32_t *hb, int *cnt) {
     using G = Geo<T>;
     constexpr int kPer = G::kRows / kConsumerWarps;
     // the warp's rows, loaded before any shared memory update (atomics and
@@ -173,59 +185,88 @@ __device__ __forceinline__ void scan_box(const uint8_t *box, int k0, int K, int 
 #pragma unroll
     for (int u = 0; u < kPer; ++u)
         vals[u] = load_elem<T>(box + (warp + u * kConsumerWarps) * G::kRowBytes + lane * (int)sizeof(T));
-    if constexpr (kKind == kScanCode) {
-        if (!ls.n_ok) return;
-        // one decision for the warp's rows: the fast codes, or the
-        // quotient's where any of them is near a rounding boundary
-        int code[kPer];
-        bool sure = true;
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            bool su;
-            code[u] = quant::quantize_fast(vals[u], ls.inv, su);
-            sure &= su;
+    for (int u = 0; u < kPer; ++u) {
+        const int k = k0 + warp + u * kConsumerWarps;
+        if (kCheck && k >= K) break;
+        const uint32_t bits = abs_bits(vals[u]);
+        if constexpr (kKind == kScanHist0) {
+            red_add_shared(&hb[bits >> (31 - kFirstBits)], 1u);
+        } else if constexpr (kKind == kScanCollect0) {
+            hb[k] = bits;
+        } else {
+            if ((bits & ls.mask) == ls.prefix) {
+                if (ls.hist) {
+                    red_add_shared(&hb[(bits >> ls.shift) & ls.dmask], 1u);
+                } else {
+                    const int j = atom_add_shared(cnt, 1);
+                    if (j < kCap) hb[j] = bits;
+                }
+            }
         }
-        if (!sure) {
+    }
+}
+
+// The code pass over one box, with the plain quantizer's thread layout: a
+// thread owns one 16-byte segment of a row (4 fp32 or 8 fp16 columns) of
+// kSweeps rows, loads each with one 16-byte read, forms the codes with one
+// exactness decision per segment and stores them as one 4- or 8-byte word.
+// Outlier split: a weight above its column's bound gets code 0 and is
+// listed (row, fp16 value) in the column's region.
+template <typename T>
+struct CodeSeg {
+    static constexpr int kCols = 16 / (int)sizeof(T);
+    static constexpr int kThreadsPerRow = kPanel / kCols;              // 8 fp32, 4 fp16
+    static constexpr int kSweep = kConsumers / kThreadsPerRow;          // 64 or 128 rows
+    static constexpr int kSweeps = Geo<T>::kRows / kSweep;              // 2
+};
+
+template <typename T, bool kCheck, bool kOut>
+__device__ __forceinline__ void code_box(const uint8_t *box, int k0, int K, int t, int rsub,
+                                         const float (&sc)[CodeSeg<T>::kCols], const float (&inv)[CodeSeg<T>::kCols],
+                                         const uint32_t (&bnd)[CodeSeg<T>::kCols], uint32_t *region, int *o_n,
+                                         int8_t *qseg, int64_t N) {
+    using S = CodeSeg<T>;
+    using G = Geo<T>;
+    float v[S::kSweeps][S::kCols];
 #pragma unroll
-            for (int u = 0; u < kPer; ++u) code[u] = quant::quantize_exact(vals[u], ls.sc);
+    for (int w = 0; w < S::kSweeps; ++w) quant::load_seg<T>(box + (rsub + w * S::kSweep) * G::kRowBytes + 16 * t, v[w]);
+#pragma unroll
+    for (int w = 0; w < S::kSweeps; ++w) {
+        const int k = k0 + rsub + w * S::kSweep;
+        if (kCheck && k >= K) break;
+        int code[S::kCols];   // codes in the low bytes
+        if (!quant::quantize_fast_seg<S::kCols>(v[w], inv, code)) {
+#pragma unroll
+            for (int e = 0; e < S::kCols; ++e) code[e] = quant::quantize_exact(v[w][e], sc[e]);
         }
+        if constexpr (kOut) {
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int k = k0 + warp + u * kConsumerWarps;
-            if (kCheck && k >= K) break;
-            if constexpr (kOut) {
-                if (abs_bits(vals[u]) > ls.bound) {   // |w| above the bound
-                    const int j = atomicAdd(on, 1);
+            for (int e = 0; e < S::kCols; ++e) {
+                if (abs_bits(v[w][e]) > bnd[e]) {   // |w| above the bound
+                    const int col = t * S::kCols + e;
+                    const int j = atom_add_shared(&o_n[col], 1);
                     if (j < kMaxOutliers) {
-                        reinterpret_cast<int32_t *>(hb)[j] = k;
-                        reinterpret_cast<uint16_t *>(hb + kMaxOutliers)[j] = __half_as_ushort(__float2half_rn(vals[u]));
+                        uint32_t *cr = region + col * kRegion;
+                        reinterpret_cast<int32_t *>(cr)[j] = k;
+                        reinterpret_cast<uint16_t *>(cr + kMaxOutliers)[j] = __half_as_ushort(__float2half_rn(v[w][e]));
                     }
-                    code[u] = 0;
+                    code[e] = 0;
                 }
             }
-            qcol[(int64_t)k * N] = (int8_t)code[u];
         }
-    } else {
+        uint32_t packed[S::kCols / 4];
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int k = k0 + warp + u * kConsumerWarps;
-            if (kCheck && k >= K) break;
-            const uint32_t bits = abs_bits(vals[u]);
-            if constexpr (kKind == kScanHist0) {
-                atomicAdd(&hb[bits >> 21], 1u);
-            } else if constexpr (kKind == kScanCollect0) {
-                hb[k] = bits;
-            } else {
-                if ((bits & ls.mask) == ls.prefix) {
-                    if (ls.hist) {
-                        atomicAdd(&hb[(bits >> ls.shift) & ls.dmask], 1u);
-                    } else {
-                        const int j = atomicAdd(cnt, 1);
-                        if (j < kCap) hb[j] = bits;
-                    }
-                }
-            }
+        for (int g = 0; g < S::kCols / 4; ++g) {
+            const uint32_t lo = __byte_perm((uint32_t)code[4 * g], (uint32_t)code[4 * g + 1], 0x0040);
+            const uint32_t hi = __byte_perm((uint32_t)code[4 * g + 2], (uint32_t)code[4 * g + 3], 0x0040);
+            packed[g] = __byte_perm(lo, hi, 0x5410);
         }
+        int8_t *dst = qseg + (int64_t)k * N;
+        if constexpr (S::kCols == 4)
+            *reinterpret_cast<uint32_t *>(dst) = packed[0];
+        else
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[S::kCols / 4 - 1]);
     }
 }
 
@@ -351,13 +392,22 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
                 ls.shift = 31 - lvl - digit_width(lvl);
                 ls.dmask = (1u << digit_width(lvl)) - 1u;
                 ls.hist = mode == kHist;
-                ls.sc = code_pass ? col_scale[lane] : 0.0f;
-                ls.inv = code_pass ? col_inv[lane] : 0.0f;
-                ls.bound = col_prefix[lane];
-                ls.n_ok = (int64_t)panel * kPanel + lane < p.N;
             }
             uint32_t *const hb = region + lane * kRegion;
-            int8_t *const qcol = p.q + (int64_t)panel * kPanel + lane;
+            // the code pass: this thread's segment and its columns' constants
+            using S = CodeSeg<T>;
+            const int st = c % S::kThreadsPerRow, srow = c / S::kThreadsPerRow;
+            float ssc[S::kCols], sinv[S::kCols];
+            uint32_t sbnd[S::kCols];
+#pragma unroll
+            for (int e = 0; e < S::kCols; ++e) {
+                ssc[e] = code_pass ? col_scale[st * S::kCols + e] : 0.0f;
+                sinv[e] = code_pass ? col_inv[st * S::kCols + e] : 0.0f;
+                sbnd[e] = col_prefix[st * S::kCols + e];
+            }
+            // N % 8 == 0: a segment is all inside the weight or all outside
+            const bool seg_ok = (int64_t)panel * kPanel + st * S::kCols < p.N;
+            int8_t *const qseg = p.q + (int64_t)panel * kPanel + st * S::kCols;
             // which form this pass takes (the same in every warp)
             const int kind = code_pass ? kScanCode : (pass > 0 ? kScanSelect : (K > kCap ? kScanHist0 : kScanCollect0));
             for (int i = 0; i < nbox; ++i) {
@@ -366,12 +416,17 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
                     const uint8_t *box = ring + s * kBoxBytes;
                     const int k0 = i * G::kRows;
                     const bool chk = k0 + G::kRows > K;
-#define W8_SCAN(KIND)                                                                                       \
-    (chk ? scan_box<T, KIND, true, kOut>(box, k0, K, warp, lane, ls, hb, &col_cnt[lane], &o_n[lane], qcol, p.N) \
-         : scan_box<T, KIND, false, kOut>(box, k0, K, warp, lane, ls, hb, &col_cnt[lane], &o_n[lane], qcol, p.N))
-                    if (kind == kScanCode)
-                        W8_SCAN(kScanCode);
-                    else if (kind == kScanSelect)
+#define W8_SCAN(KIND)                                                                       \
+    (chk ? scan_box<T, KIND, true, kOut>(box, k0, K, warp, lane, ls, hb, &col_cnt[lane]) \
+         : scan_box<T, KIND, false, kOut>(box, k0, K, warp, lane, ls, hb, &col_cnt[lane]))
+                    if (kind == kScanCode) {
+                        if (seg_ok) {
+                            if (chk)
+                                code_box<T, true, kOut>(box, k0, K, st, srow, ssc, sinv, sbnd, region, o_n, qseg, p.N);
+                            else
+                                code_box<T, false, kOut>(box, k0, K, st, srow, ssc, sinv, sbnd, region, o_n, qseg, p.N);
+                        }
+                    } else if (kind == kScanSelect)
                         W8_SCAN(kScanSelect);
                     else if (kind == kScanHist0)
                         W8_SCAN(kScanHist0);
@@ -443,7 +498,7 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
                     uint32_t *const sb = scratch + warp * kScratch;
 #pragma unroll 1
                     while (clvl < 31) {
-                        const int w = digit_width(clvl == 0 ? 1 : clvl);   // 7-bit digits here
+                        const int w = collect_width(clvl);
                         const int sh = 31 - clvl - w;
                         const uint32_t m = prefix_mask(clvl);
                         for (int b = lane; b < (1 << w); b += 32) sb[b] = 0u;
