@@ -136,9 +136,11 @@ int w8_quantize_per_channel_asym(const void *W, int w_dtype, int64_t K, int64_t 
  * -127, 127 ) as in w8_quantize_per_channel: weights beyond the bound land on
  * +-127.  The output is in the symmetric format (w8_prepack, w8a16_linear).
  * c = +inf and p = 1 give w8_quantize_per_channel's result bit for bit.
- * The percentile form finds the order statistic by a four-pass radix
- * selection on the bit patterns of |w| and streams W five times (the passes
- * after the first mostly from L2).
+ * The percentile form finds the order statistic by radix selection on the
+ * bit patterns of |w| (digits of 9, 8, 7 and 7 bits; a column's last
+ * candidates, at most 768, are selected in shared memory) and streams W
+ * three times for usual weights, at most five times (the passes after the
+ * first mostly from L2).
  * Errors: as w8_quantize_per_channel; W8_ERR_SHAPE also for a clip_param
  * out of range, W8_ERR_DTYPE for an unknown clip_mode.
  */
