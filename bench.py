@@ -231,6 +231,8 @@ def replay_times(graph, reps, stream, ws, device, sampler):
 # loop under the power cap.  A timed region shorter than SUSTAINED_S is
 # compared with the burst figure.
 SUSTAINED_S = 2.0
+# Idle time before the variants' prefill timings (see there).
+IDLE_S = 2.0
 
 
 def tensor_peak(region_s, tf_peak, tf_sustained):
@@ -457,15 +459,22 @@ def run_native(args, ws, rank, local):
         torch.cuda.empty_cache()
 
     # ---- the variants' prefill calls (M = 2048), each timed as the plain
-    # call is (a graph of two calls, back to back), with the plain call timed
-    # just before them so that the ratios compare like with like; before the
-    # long prefill loop, after which the outlier split's memory-bound parts
-    # measured slower (523 against 441 us)
+    # call is (a graph of two calls, back to back) and, like the plain call
+    # timed for them, from an idle GPU: after seconds of power-capped tensor
+    # work the outlier split's call measured up to 37 % slower (440 -> 602
+    # us) and the plain call 17 % (298 -> 349 us), and two idle seconds
+    # brought both back
     if not args.no_variants:
         fl_pf = 2.0 * M_PREFILL * K_DIM * N_DIM
-        t_plain = graph_time(lambda: [w8.linear(Xp, c, scales, out=Yp) for c in copies[:2]], 20) / 2
-        t_pa = graph_time(lambda: [w8.linear_asym(Xp, c, sa, za, out=Yp) for c in pa], 20) / 2
-        t_po = graph_time(lambda: [w8.linear_outliers(Xp, c, so, co, ro, vo, out=Yp) for c in po], 20) / 2
+
+        def from_idle(fn):
+            torch.cuda.synchronize()
+            time.sleep(IDLE_S)
+            return graph_time(fn, 20) / 2
+
+        t_plain = from_idle(lambda: [w8.linear(Xp, c, scales, out=Yp) for c in copies[:2]])
+        t_pa = from_idle(lambda: [w8.linear_asym(Xp, c, sa, za, out=Yp) for c in pa])
+        t_po = from_idle(lambda: [w8.linear_outliers(Xp, c, so, co, ro, vo, out=Yp) for c in po])
         variants["asymmetric"].update({
             "prefill_m2048_us": round(t_pa * 1e6, 1), "prefill_m2048_TFLOPs": round(fl_pf / t_pa / 1e12, 1),
             "prefill_m2048_frac_tensor_burst": round(fl_pf / t_pa / 1e12 / tf_peak, 4),
@@ -475,6 +484,7 @@ def run_native(args, ws, rank, local):
             "prefill_m2048_frac_tensor_burst": round(fl_pf / t_po / 1e12 / tf_peak, 4),
             "prefill_m2048_vs_plain": round(t_po / t_plain, 3)})
         variants["prefill_m2048_plain_us_alongside"] = round(t_plain * 1e6, 1)
+        variants["prefill_m2048_timed_from"] = f"an idle GPU ({IDLE_S} s before each of the three)"
         del pa, po
         torch.cuda.empty_cache()
 
