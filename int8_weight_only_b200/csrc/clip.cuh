@@ -496,6 +496,26 @@ percentile_quantize_kernel(const __grid_constant__ CUtensorMap tmap_w, const Par
                     // histogram goes to the warp's scratch
                     const int cnt = min(col_cnt[col], kCap);
                     uint32_t *const sb = scratch + warp * kScratch;
+                    if (cnt <= 32) {
+                        // one pattern per lane: the wanted one has fewer than rem
+                        // patterns above it and at least rem at or above it
+                        const uint32_t x = lane < cnt ? cb[lane] : 0u;
+                        uint32_t above = 0, same = 0;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const uint32_t y = __shfl_sync(0xffffffffu, x, j);
+                            if (j < cnt) {
+                                above += y > x;
+                                same += y == x;
+                            }
+                        }
+                        const uint32_t hit = __ballot_sync(0xffffffffu, lane < cnt && above < rem && rem <= above + same);
+                        const int src = hit ? __ffs(hit) - 1 : 0;
+                        pre = __shfl_sync(0xffffffffu, x, src);
+                        rem -= __shfl_sync(0xffffffffu, above, src);
+                        grp = __shfl_sync(0xffffffffu, same, src);
+                        clvl = 31;
+                    }
 #pragma unroll 1
                     while (clvl < 31) {
                         const int w = collect_width(clvl);
