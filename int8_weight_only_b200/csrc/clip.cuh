@@ -15,8 +15,9 @@
 //  - histogram: count the values with the prefix by their next digit; the
 //    bin that holds the wanted rank extends the prefix;
 //  - collect: once at most kCap values carry the prefix, copy their
-//    patterns into shared memory, and finish the selection there (digit
-//    by digit again, within one warp, with no further pass over W).
+//    patterns into shared memory, and finish the selection there within
+//    one warp, with no further pass over W (up to 32 patterns: one per
+//    lane, ranked by a count over warp shuffles; more: digit by digit).
 // On the usual weights the first pass (a 512-bin histogram) leaves a few
 // values in the chosen bin, the second collects them and the third writes
 // the codes: three passes over W instead of the five a byte-wise radix
